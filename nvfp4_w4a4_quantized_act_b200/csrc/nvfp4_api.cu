@@ -1,0 +1,522 @@
+// nvfp4_api.cu -- the C ABI of libnvfp4.so: argument checks, workspace
+// carving, TMA descriptor set-up and kernel launches for the NVFP4 W4A4
+// linear layer.  Every entry point is declared and documented in
+// include/nvfp4.h.
+#include <atomic>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "nvfp4.h"
+#include "gemm_kernel.cuh"
+#include "quantize_kernels.cuh"
+
+namespace {
+
+using nvfp4::kMaxSeg;
+
+__device__ uint32_t g_status_word;  // per-device latched error bits
+
+std::atomic<uint64_t> g_launches{0};
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceState {
+    bool init = false;
+    bool supported = false;
+    int sm_count = 0;
+    uint32_t *status = nullptr;  // device address of g_status_word
+    bool gemm_attr_set = false;
+};
+
+DeviceState g_dev[kMaxDevices];
+std::mutex g_mu;
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+
+// Looks up (once per device) the SM count, the status word address and
+// whether the device is an sm_100 part.  Returns nullptr on failure.
+DeviceState *device_state()
+{
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+        return nullptr;
+    DeviceState &d = g_dev[dev];
+    if (d.init)
+        return &d;
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (d.init)
+        return &d;
+    cudaDeviceProp prop;
+    if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess)
+        return nullptr;
+    d.supported = (prop.major == 10 && prop.minor == 0);
+    d.sm_count = prop.multiProcessorCount;
+    if (d.supported) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess)
+            return nullptr;
+        d.status = static_cast<uint32_t *>(p);
+        if (cudaFuncSetAttribute(nvfp4::gemm::gemm_nvf4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 nvfp4::gemm::SMEM_BYTES) != cudaSuccess)
+            return nullptr;
+        d.gemm_attr_set = true;
+        if (g_encode == nullptr) {
+            void *fn = nullptr;
+            cudaDriverEntryPointQueryResult q;
+            if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+                q != cudaDriverEntryPointSuccess || fn == nullptr)
+                return nullptr;
+            g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+        }
+    }
+    d.init = true;
+    return &d;
+}
+
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline int64_t round_up(int64_t a, int64_t b) { return (a + b - 1) / b * b; }
+inline int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+int64_t sf_bytes_i(int64_t rows, int64_t K) { return round_up(rows, 128) * cdiv(K / 16, 4) * 4; }
+
+int check_segments(const nvfp4_segment *segs, int nseg, int64_t N, nvfp4::SegRows *out)
+{
+    if (segs == nullptr || nseg < 1 || nseg > kMaxSeg)
+        return NVFP4_ERR_INVALID_ARG;
+    int64_t expect = 0;
+    out->nseg = nseg;
+    for (int i = 0; i < nseg; ++i) {
+        if (segs[i].n_begin != expect || segs[i].n_end < segs[i].n_begin)
+            return NVFP4_ERR_INVALID_ARG;
+        expect = segs[i].n_end;
+        out->end[i] = segs[i].n_end;
+    }
+    for (int i = nseg; i < kMaxSeg; ++i)
+        out->end[i] = N;
+    return expect == N ? NVFP4_OK : NVFP4_ERR_INVALID_ARG;
+}
+
+int launch_ok()
+{
+    return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
+}
+
+// K1 + K2 for `rows` x K bf16 rows, segment table `seg`.  mode 0: dynamic
+// scale from max|x| (amax words in ws, g written to g_out); mode 1: scale
+// read from g_in.
+int run_quantize(DeviceState *d, const void *X, int64_t rows, int64_t K, int64_t ld, const nvfp4::SegRows &seg,
+                 uint8_t *codes, uint8_t *sf, const float *g_in, float *g_out, bool dynamic, uint32_t *amax_ws,
+                 cudaStream_t stream)
+{
+    const int64_t rows_pad = round_up(rows, 128);
+    const int64_t groups = cdiv(K, 64);
+    if (rows_pad * groups * 4 >= (int64_t(1) << 31) || K > (int64_t(1) << 30))
+        return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (dynamic) {
+        if (cudaMemsetAsync(amax_ws, 0, sizeof(uint32_t) * seg.nseg, stream) != cudaSuccess)
+            return NVFP4_ERR_CUDA;
+        g_launches++;
+        if (rows > 0) {
+            const int64_t warps_needed = rows;
+            int grid = static_cast<int>(std::min<int64_t>(cdiv(warps_needed, 8), int64_t(d->sm_count) * 8));
+            nvfp4::amax_kernel<<<grid, 256, 0, stream>>>(static_cast<const uint16_t *>(X), rows, K, ld, seg,
+                                                          amax_ws, d->status);
+            g_launches++;
+            if (launch_ok() != NVFP4_OK)
+                return NVFP4_ERR_CUDA;
+        }
+    }
+    nvfp4::QuantParams p;
+    p.X = static_cast<const uint16_t *>(X);
+    p.ld = ld;
+    p.rows = static_cast<int32_t>(rows);
+    p.K = static_cast<int32_t>(K);
+    p.rows_pad = static_cast<int32_t>(rows_pad);
+    p.groups = static_cast<int32_t>(groups);
+    p.seg = seg;
+    p.amax_bits = amax_ws;
+    p.g_in = g_in;
+    p.g_out = g_out;
+    p.mode = dynamic ? 0 : 1;
+    p.codes = codes;
+    p.sf = sf;
+    const int64_t threads = rows_pad * groups * 4;
+    int grid = static_cast<int>(std::min<int64_t>(std::max<int64_t>(cdiv(threads, 256), 1), int64_t(d->sm_count) * 16));
+    nvfp4::quantize_kernel<<<grid, 256, 0, stream>>>(p);
+    g_launches++;
+    return launch_ok();
+}
+
+int make_codes_map(CUtensorMap *map, const uint8_t *codes, int64_t rows, int64_t K, uint32_t box_rows)
+{
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(K / 2), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(K / 2)};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(nvfp4::gemm::BK_BYTES), box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(codes), dims, strides, box,
+                          estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? NVFP4_OK : NVFP4_ERR_CUDA;
+}
+
+int run_gemm(DeviceState *d, const uint8_t *a_codes, const uint8_t *a_sf, const float *g_a, int64_t M, int64_t K,
+             const uint8_t *w_codes, const uint8_t *w_sf, int64_t N, const nvfp4::SegRows &seg, const float *g_w,
+             void *out, unsigned flags, cudaStream_t stream)
+{
+    using namespace nvfp4::gemm;
+    if (M == 0 || N == 0)
+        return NVFP4_OK;
+    CUtensorMap tmA, tmB;
+    if (make_codes_map(&tmA, a_codes, M, K, BM) != NVFP4_OK || make_codes_map(&tmB, w_codes, N, K, BN) != NVFP4_OK)
+        return NVFP4_ERR_CUDA;
+    Params p;
+    std::memset(&p, 0, sizeof(p));
+    p.M = static_cast<int32_t>(M);
+    p.N = static_cast<int32_t>(N);
+    p.K = static_cast<int32_t>(K);
+    p.num_m = static_cast<int32_t>(cdiv(M, BM));
+    p.num_n = static_cast<int32_t>(cdiv(N, BN));
+    p.num_tiles = p.num_m * p.num_n;
+    p.kb_total = static_cast<int32_t>(K / 64);
+    p.kt_total = static_cast<int32_t>(cdiv(K / 64, KB_PER_STAGE));
+    p.n_row_tiles = static_cast<int32_t>(cdiv(N, 128));
+    p.sfa = a_sf;
+    p.sfb = w_sf;
+    p.g_a = g_a;
+    p.g_w = g_w;
+    p.nseg = seg.nseg;
+    for (int i = 0; i < kMaxSeg; ++i)
+        p.seg_end[i] = static_cast<int32_t>(seg.end[i]);
+    p.out = out;
+    p.out_fp32 = (flags & NVFP4_OUT_FP32) ? 1 : 0;
+    const int64_t esz = p.out_fp32 ? 4 : 2;
+    p.vec_ok = aligned16(out) && ((N * esz) % 16 == 0);
+    p.status = d->status;
+    const int grid = static_cast<int>(std::min<int64_t>(p.num_tiles, d->sm_count));
+    gemm_nvf4_kernel<<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(tmA, tmB, p);
+    g_launches++;
+    return launch_ok();
+}
+
+int check_gemm_shape(int64_t M, int64_t N, int64_t K)
+{
+    if (M < 0 || N < 0 || K <= 0)
+        return NVFP4_ERR_INVALID_ARG;
+    if (K % 64 != 0)
+        return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (M > (int64_t(1) << 30) || N > (int64_t(1) << 30) || K > (int64_t(1) << 30) ||
+        cdiv(M, 128) * cdiv(N, 192) >= (int64_t(1) << 31))
+        return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    return NVFP4_OK;
+}
+
+constexpr size_t kLinScaleOff = 256;
+constexpr size_t kLinCodesOff = 1024;
+
+size_t linear_codes_bytes(int64_t M, int64_t K) { return static_cast<size_t>(M) * static_cast<size_t>(K / 2); }
+
+size_t linear_sf_off(int64_t M, int64_t K)
+{
+    return static_cast<size_t>(round_up(static_cast<int64_t>(kLinCodesOff + linear_codes_bytes(M, K)), 1024));
+}
+
+}  // namespace
+
+// ======================================================================== C ABI
+
+extern "C" {
+
+size_t nvfp4_sf_bytes(int64_t rows, int64_t K)
+{
+    if (rows < 0 || K <= 0 || K % 16 != 0)
+        return 0;
+    return static_cast<size_t>(sf_bytes_i(rows, K));
+}
+
+size_t nvfp4_quant_workspace_bytes(int nseg)
+{
+    if (nseg < 1 || nseg > kMaxSeg)
+        return 0;
+    return 256;
+}
+
+size_t nvfp4_workspace_bytes(int64_t M, int64_t N, int64_t K, int nseg)
+{
+    (void)N;
+    (void)nseg;
+    if (M < 0 || K <= 0 || K % 16 != 0)
+        return 0;
+    return linear_sf_off(M, K) + static_cast<size_t>(sf_bytes_i(M, K));
+}
+
+size_t nvfp4_linear_act_scale_offset(void) { return kLinScaleOff; }
+
+int nvfp4_quantize_weights(const void *W, int64_t N, int64_t K, int64_t ldw, const nvfp4_segment *segs, int nseg,
+                           uint8_t *codes, uint8_t *sf, float *g_w, void *ws, size_t ws_bytes, void *stream)
+{
+    if (g_w == nullptr || N < 0 || K <= 0 || (N > 0 && (W == nullptr || codes == nullptr || sf == nullptr)))
+        return NVFP4_ERR_INVALID_ARG;
+    if (K % 16 != 0)
+        return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (ldw < K)
+        return NVFP4_ERR_INVALID_ARG;
+    if (!aligned16(W) || ldw % 8 != 0 || !aligned16(codes) || !aligned16(sf))
+        return NVFP4_ERR_MISALIGNED;
+    nvfp4::SegRows seg;
+    int rc = check_segments(segs, nseg, N, &seg);
+    if (rc != NVFP4_OK)
+        return rc;
+    if (ws == nullptr || ws_bytes < nvfp4_quant_workspace_bytes(nseg))
+        return NVFP4_ERR_WORKSPACE;
+    DeviceState *d = device_state();
+    if (d == nullptr)
+        return NVFP4_ERR_CUDA;
+    if (!d->supported)
+        return NVFP4_ERR_NO_DEVICE;
+    return run_quantize(d, W, N, K, ldw, seg, codes, sf, nullptr, g_w, true, static_cast<uint32_t *>(ws),
+                        static_cast<cudaStream_t>(stream));
+}
+
+int nvfp4_quantize_act(const void *X, int64_t M, int64_t K, int64_t ldx, uint8_t *codes, uint8_t *sf, float *g_a,
+                       unsigned flags, void *ws, size_t ws_bytes, void *stream)
+{
+    if (g_a == nullptr || M < 0 || K <= 0 || (M > 0 && (X == nullptr || codes == nullptr || sf == nullptr)))
+        return NVFP4_ERR_INVALID_ARG;
+    if ((flags & ~(NVFP4_STATIC_SCALE | NVFP4_OUT_FP32)) != 0)
+        return NVFP4_ERR_INVALID_ARG;
+    if (K % 16 != 0)
+        return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (ldx < K)
+        return NVFP4_ERR_INVALID_ARG;
+    if (!aligned16(X) || ldx % 8 != 0 || !aligned16(codes) || !aligned16(sf) ||
+        (reinterpret_cast<uintptr_t>(g_a) & 3u))
+        return NVFP4_ERR_MISALIGNED;
+    const bool dynamic = (flags & NVFP4_STATIC_SCALE) == 0;
+    if (dynamic && (ws == nullptr || ws_bytes < nvfp4_quant_workspace_bytes(1)))
+        return NVFP4_ERR_WORKSPACE;
+    DeviceState *d = device_state();
+    if (d == nullptr)
+        return NVFP4_ERR_CUDA;
+    if (!d->supported)
+        return NVFP4_ERR_NO_DEVICE;
+    nvfp4::SegRows seg;
+    nvfp4_segment one = {0, M};
+    check_segments(&one, 1, M, &seg);
+    return run_quantize(d, X, M, K, ldx, seg, codes, sf, g_a, g_a, dynamic, static_cast<uint32_t *>(ws),
+                        static_cast<cudaStream_t>(stream));
+}
+
+int nvfp4_gemm_prequant(const uint8_t *a_codes, const uint8_t *a_sf, const float *g_a, int64_t M, int64_t K,
+                        const uint8_t *w_codes, const uint8_t *w_sf, int64_t N, const nvfp4_segment *segs,
+                        const float *g_w, int nseg, void *out, unsigned flags, void *stream)
+{
+    if ((flags & ~(NVFP4_STATIC_SCALE | NVFP4_OUT_FP32)) != 0)
+        return NVFP4_ERR_INVALID_ARG;
+    int rc = check_gemm_shape(M, N, K);
+    if (rc != NVFP4_OK)
+        return rc;
+    {
+        nvfp4::SegRows seg0;
+        rc = check_segments(segs, nseg, N, &seg0);
+        if (rc != NVFP4_OK)
+            return rc;
+    }
+    if (M == 0 || N == 0)
+        return NVFP4_OK;
+    if (a_codes == nullptr || a_sf == nullptr || g_a == nullptr || w_codes == nullptr || w_sf == nullptr ||
+        g_w == nullptr || out == nullptr)
+        return NVFP4_ERR_INVALID_ARG;
+    if (!aligned16(a_codes) || !aligned16(a_sf) || !aligned16(w_codes) || !aligned16(w_sf) ||
+        (reinterpret_cast<uintptr_t>(g_a) & 3u) || (reinterpret_cast<uintptr_t>(g_w) & 3u) ||
+        (reinterpret_cast<uintptr_t>(out) & ((flags & NVFP4_OUT_FP32) ? 3u : 1u)))
+        return NVFP4_ERR_MISALIGNED;
+    nvfp4::SegRows seg;
+    rc = check_segments(segs, nseg, N, &seg);
+    if (rc != NVFP4_OK)
+        return rc;
+    DeviceState *d = device_state();
+    if (d == nullptr)
+        return NVFP4_ERR_CUDA;
+    if (!d->supported)
+        return NVFP4_ERR_NO_DEVICE;
+    return run_gemm(d, a_codes, a_sf, g_a, M, K, w_codes, w_sf, N, seg, g_w, out, flags,
+                    static_cast<cudaStream_t>(stream));
+}
+
+int nvfp4_linear_fused(const void *X, int64_t M, int64_t K, const uint8_t *w_codes, const uint8_t *w_sf, int64_t N,
+                       const nvfp4_segment *segs, const float *g_w, int nseg, void *out, unsigned flags, void *ws,
+                       size_t ws_bytes, void *stream)
+{
+    if ((flags & ~(NVFP4_STATIC_SCALE | NVFP4_OUT_FP32)) != 0)
+        return NVFP4_ERR_INVALID_ARG;
+    int rc = check_gemm_shape(M, N, K);
+    if (rc != NVFP4_OK)
+        return rc;
+    {
+        nvfp4::SegRows seg0;
+        rc = check_segments(segs, nseg, N, &seg0);
+        if (rc != NVFP4_OK)
+            return rc;
+    }
+    if (M == 0 || N == 0)
+        return NVFP4_OK;
+    if (X == nullptr || w_codes == nullptr || w_sf == nullptr || g_w == nullptr || out == nullptr)
+        return NVFP4_ERR_INVALID_ARG;
+    if (!aligned16(X) || K % 8 != 0 || !aligned16(w_codes) || !aligned16(w_sf) ||
+        (reinterpret_cast<uintptr_t>(g_w) & 3u) ||
+        (reinterpret_cast<uintptr_t>(out) & ((flags & NVFP4_OUT_FP32) ? 3u : 1u)))
+        return NVFP4_ERR_MISALIGNED;
+    nvfp4::SegRows seg;
+    rc = check_segments(segs, nseg, N, &seg);
+    if (rc != NVFP4_OK)
+        return rc;
+    if (ws == nullptr || !aligned16(ws) || ws_bytes < nvfp4_workspace_bytes(M, N, K, nseg))
+        return NVFP4_ERR_WORKSPACE;
+    DeviceState *d = device_state();
+    if (d == nullptr)
+        return NVFP4_ERR_CUDA;
+    if (!d->supported)
+        return NVFP4_ERR_NO_DEVICE;
+    uint8_t *base = static_cast<uint8_t *>(ws);
+    uint32_t *amax = reinterpret_cast<uint32_t *>(base);
+    float *g_a = reinterpret_cast<float *>(base + kLinScaleOff);
+    uint8_t *a_codes = base + kLinCodesOff;
+    uint8_t *a_sf = base + linear_sf_off(M, K);
+    nvfp4::SegRows one_seg;
+    nvfp4_segment one = {0, M};
+    check_segments(&one, 1, M, &one_seg);
+    const bool dynamic = (flags & NVFP4_STATIC_SCALE) == 0;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    rc = run_quantize(d, X, M, K, K, one_seg, a_codes, a_sf, g_a, g_a, dynamic, amax, s);
+    if (rc != NVFP4_OK)
+        return rc;
+    return run_gemm(d, a_codes, a_sf, g_a, M, K, w_codes, w_sf, N, seg, g_w, out, flags, s);
+}
+
+int nvfp4_linear(const void *X, int64_t M, int64_t K, const uint8_t *w_codes, const uint8_t *w_sf, const float *g_w,
+                 int64_t N, void *out, unsigned flags, void *ws, size_t ws_bytes, void *stream)
+{
+    if (N < 0)
+        return NVFP4_ERR_INVALID_ARG;
+    nvfp4_segment one = {0, N};
+    return nvfp4_linear_fused(X, M, K, w_codes, w_sf, N, &one, g_w, 1, out, flags, ws, ws_bytes, stream);
+}
+
+int nvfp4_swiglu_quantize(const void *gate_up, int64_t M, int64_t F, int64_t ld, void *h, uint8_t *codes, uint8_t *sf,
+                          float *g_h, void *ws, size_t ws_bytes, void *stream)
+{
+    if (gate_up == nullptr || h == nullptr || codes == nullptr || sf == nullptr || g_h == nullptr || M < 0 || F <= 0)
+        return NVFP4_ERR_INVALID_ARG;
+    if (F % 16 != 0)
+        return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (ld < 2 * F)
+        return NVFP4_ERR_INVALID_ARG;
+    if (!aligned16(gate_up) || ld % 8 != 0 || !aligned16(h) || !aligned16(codes) || !aligned16(sf))
+        return NVFP4_ERR_MISALIGNED;
+    if (ws == nullptr || ws_bytes < nvfp4_quant_workspace_bytes(1))
+        return NVFP4_ERR_WORKSPACE;
+    if (M * (F / 8) >= (int64_t(1) << 31))
+        return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    DeviceState *d = device_state();
+    if (d == nullptr)
+        return NVFP4_ERR_CUDA;
+    if (!d->supported)
+        return NVFP4_ERR_NO_DEVICE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint32_t *amax = static_cast<uint32_t *>(ws);
+    if (cudaMemsetAsync(amax, 0, sizeof(uint32_t), s) != cudaSuccess)
+        return NVFP4_ERR_CUDA;
+    g_launches++;
+    if (M > 0) {
+        const int64_t threads = M * (F / 8);
+        const int grid = static_cast<int>(std::min<int64_t>(cdiv(threads, 256), int64_t(d->sm_count) * 16));
+        nvfp4::swiglu_kernel<<<grid, 256, 0, s>>>(static_cast<const uint16_t *>(gate_up), ld,
+                                                  static_cast<int32_t>(M), static_cast<int32_t>(F),
+                                                  static_cast<uint16_t *>(h), amax);
+        g_launches++;
+        if (launch_ok() != NVFP4_OK)
+            return NVFP4_ERR_CUDA;
+    }
+    nvfp4::SegRows seg;
+    nvfp4_segment one = {0, M};
+    check_segments(&one, 1, M, &seg);
+    // the amax of h was folded in by the SwiGLU kernel: quantize without a new amax pass
+    const int64_t rows_pad = round_up(M, 128);
+    const int64_t groups = cdiv(F, 64);
+    if (rows_pad * groups * 4 >= (int64_t(1) << 31))
+        return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    nvfp4::QuantParams p;
+    p.X = static_cast<const uint16_t *>(h);
+    p.ld = F;
+    p.rows = static_cast<int32_t>(M);
+    p.K = static_cast<int32_t>(F);
+    p.rows_pad = static_cast<int32_t>(rows_pad);
+    p.groups = static_cast<int32_t>(groups);
+    p.seg = seg;
+    p.amax_bits = amax;
+    p.g_in = nullptr;
+    p.g_out = g_h;
+    p.mode = 0;
+    p.codes = codes;
+    p.sf = sf;
+    const int64_t threads = rows_pad * groups * 4;
+    const int grid = static_cast<int>(std::min<int64_t>(std::max<int64_t>(cdiv(threads, 256), 1), int64_t(d->sm_count) * 16));
+    nvfp4::quantize_kernel<<<grid, 256, 0, s>>>(p);
+    g_launches++;
+    return launch_ok();
+}
+
+int nvfp4_get_status(void *stream)
+{
+    DeviceState *d = device_state();
+    if (d == nullptr)
+        return NVFP4_ERR_CUDA;
+    if (!d->supported)
+        return NVFP4_ERR_NO_DEVICE;
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return NVFP4_ERR_CUDA;
+    uint32_t v = 0;
+    if (cudaMemcpy(&v, d->status, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return NVFP4_ERR_CUDA;
+    const uint32_t zero = 0;
+    if (cudaMemcpy(d->status, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess)
+        return NVFP4_ERR_CUDA;
+    if (v & nvfp4::kStatusTimeout)
+        return NVFP4_ERR_TIMEOUT;
+    if (v & nvfp4::kStatusNonFinite)
+        return NVFP4_ERR_NONFINITE;
+    return NVFP4_OK;
+}
+
+const char *nvfp4_status_string(int status)
+{
+    switch (status) {
+    case NVFP4_OK: return "ok";
+    case NVFP4_ERR_INVALID_ARG: return "invalid argument";
+    case NVFP4_ERR_UNSUPPORTED_SHAPE: return "unsupported shape (K must be a multiple of 16, 64 for GEMMs)";
+    case NVFP4_ERR_MISALIGNED: return "misaligned pointer or leading dimension";
+    case NVFP4_ERR_CUDA: return "CUDA runtime error";
+    case NVFP4_ERR_TIMEOUT: return "a bounded wait inside a kernel ran out";
+    case NVFP4_ERR_NONFINITE: return "input contains Inf or NaN";
+    case NVFP4_ERR_WORKSPACE: return "workspace missing or too small";
+    case NVFP4_ERR_NO_DEVICE: return "current device is not an sm_100 GPU";
+    default: return "unknown status";
+    }
+}
+
+int nvfp4_device_supported(void)
+{
+    DeviceState *d = device_state();
+    return (d != nullptr && d->supported) ? 1 : 0;
+}
+
+uint64_t nvfp4_launch_count(void) { return g_launches.load(); }
+
+}  // extern "C"

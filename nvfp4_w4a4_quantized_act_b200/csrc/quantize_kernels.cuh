@@ -1,0 +1,264 @@
+// quantize_kernels.cuh -- HBM-bound NVFP4 codec kernels for sm_100a.
+//
+//  amax_kernel      max|x| per module segment (per tensor for activations):
+//                   one warp per row, 16-byte loads, packed 16-bit integer
+//                   max of bf16 magnitudes (non-negative floats order like
+//                   their bit patterns), one shared then one global atomic
+//                   per CTA and segment.
+//  quantize_kernel  per 16-element block: E4M3 scale and E2M1 codes, two
+//                   codes per byte, scales written straight into the 128x4
+//                   tile layout the block-scaled MMA reads (four neighbouring
+//                   blocks of a row form one 32-bit word, gathered by warp
+//                   shuffles).
+//  swiglu_kernel    h = bf16(silu(gate) * up) for a fused gate/up output, plus
+//                   max|h| for its dynamic global scale.
+//
+// Format and scale conventions: NVFP4 = E2M1 values with an E4M3 scale per
+// 16-element block ("NVFP4 W4A4 quantization compresses 27B hybrid models",
+// thevalue.engineering, "Challenging the Recurrence Fragility Assumption"),
+// one FP32 global scale per calibrated module ("Why Gated DeltaNet Survives
+// 4-Bit Quantization", kipquest.com, "The abstract").
+#pragma once
+
+#include <cstdint>
+#include <cuda_bf16.h>
+
+#include "ptx_sm100.cuh"
+
+namespace nvfp4 {
+
+constexpr int kMaxSeg = 16;
+constexpr uint32_t kStatusTimeout = 1u;
+constexpr uint32_t kStatusNonFinite = 2u;
+
+// Rows [0, end[0]) belong to segment 0, [end[i-1], end[i]) to segment i.
+struct SegRows {
+    int32_t nseg;
+    int64_t end[kMaxSeg];
+};
+
+__device__ __forceinline__ int seg_of(const SegRows &s, int64_t r)
+{
+    int k = 0;
+#pragma unroll 1
+    while (k + 1 < s.nseg && r >= s.end[k])
+        ++k;
+    return k;
+}
+
+// Packed max of the magnitudes (sign cleared) of the two bf16 in `w`.
+__device__ __forceinline__ uint32_t vmax_mag(uint32_t acc, uint32_t w)
+{
+    return __vmaxu2(acc, w & 0x7FFF7FFFu);
+}
+
+__device__ __forceinline__ uint32_t vmax_mag(uint32_t acc, const uint4 &v)
+{
+    acc = vmax_mag(acc, v.x);
+    acc = vmax_mag(acc, v.y);
+    acc = vmax_mag(acc, v.z);
+    acc = vmax_mag(acc, v.w);
+    return acc;
+}
+
+__device__ __forceinline__ uint32_t hmax16(uint32_t packed) { return max(packed & 0xFFFFu, packed >> 16); }
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// ------------------------------------------------------------------ amax
+
+// amax_bits[seg] = max over the segment's rows of the bf16 magnitude bits
+// (the float max|x| is amax_bits << 16).  amax_bits must be zero on entry.
+__global__ void __launch_bounds__(256) amax_kernel(const uint16_t *__restrict__ X, int64_t rows, int64_t K,
+                                                   int64_t ld, SegRows seg, uint32_t *__restrict__ amax_bits,
+                                                   uint32_t *__restrict__ status)
+{
+    __shared__ uint32_t s_max[kMaxSeg];
+    if (threadIdx.x < kMaxSeg)
+        s_max[threadIdx.x] = 0;
+    __syncthreads();
+
+    const int lane = threadIdx.x & 31;
+    const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+    const int64_t chunks = K >> 3;  // 16-byte chunks per row
+
+    int slot = 0;
+    uint32_t m = 0;
+    for (int64_t r = warp; r < rows; r += nwarps) {
+        const int s = seg_of(seg, r);
+        if (s != slot) {  // warp-uniform: every lane works on row r
+            atomicMax(&s_max[slot], hmax16(m));
+            m = 0;
+            slot = s;
+        }
+        const uint4 *p = reinterpret_cast<const uint4 *>(X + r * ld);
+        int64_t j = lane;
+        for (; j + 96 < chunks; j += 128) {
+            const uint4 a = __ldg(p + j), b = __ldg(p + j + 32), c = __ldg(p + j + 64), d = __ldg(p + j + 96);
+            m = vmax_mag(m, a);
+            m = vmax_mag(m, b);
+            m = vmax_mag(m, c);
+            m = vmax_mag(m, d);
+        }
+        for (; j < chunks; j += 32)
+            m = vmax_mag(m, __ldg(p + j));
+    }
+    atomicMax(&s_max[slot], hmax16(m));
+    __syncthreads();
+    if (threadIdx.x < seg.nseg) {
+        const uint32_t v = s_max[threadIdx.x];
+        if (v != 0)
+            atomicMax(&amax_bits[threadIdx.x], v);
+        if (v >= 0x7F80u)  // Inf or NaN magnitude
+            atomicOr(status, kStatusNonFinite);
+    }
+}
+
+// ------------------------------------------------------------- quantize
+
+struct QuantParams {
+    const uint16_t *X;       // bf16 [rows, K], leading dimension ld
+    int64_t ld;
+    int32_t rows;
+    int32_t K;
+    int32_t rows_pad;        // rows rounded up to 128
+    int32_t groups;          // ceil(K / 64): 32-bit scale words per row
+    SegRows seg;
+    const uint32_t *amax_bits;  // mode 0: per-segment amax bits
+    const float *g_in;          // mode 1: per-segment global scale
+    float *g_out;               // mode 0: per-segment global scale written here (may be null)
+    int32_t mode;
+    uint8_t *codes;          // [rows, K/2]
+    uint8_t *sf;             // swizzled scale tiles
+};
+
+__device__ __forceinline__ float global_scale_from_amax(uint32_t bits)
+{
+    const float a = __uint_as_float(bits << 16);
+    return a == 0.0f ? 1.0f : __fdiv_rn(a, 2688.0f);
+}
+
+// One thread per 16-element block; four consecutive threads cover the four
+// blocks that share one 32-bit scale word.  Grid-stride over
+// rows_pad * groups * 4 threads (rows past `rows` only write zero scales).
+__global__ void __launch_bounds__(256) quantize_kernel(const QuantParams p)
+{
+    const uint32_t total = static_cast<uint32_t>(p.rows_pad) * static_cast<uint32_t>(p.groups) * 4u;
+    const uint32_t stride = gridDim.x * blockDim.x;
+    const int lane = threadIdx.x & 31;
+    const int nblk = p.K >> 4;
+
+    if (p.mode == 0 && p.g_out != nullptr && blockIdx.x == 0 && threadIdx.x < p.seg.nseg)
+        p.g_out[threadIdx.x] = global_scale_from_amax(p.amax_bits[threadIdx.x]);
+
+    // Loop bound is warp-uniform so every lane takes part in the shuffles.
+    for (uint32_t base = blockIdx.x * blockDim.x + (threadIdx.x & ~31u); base < total; base += stride) {
+        const uint32_t t = base + lane;
+        const uint32_t u = t >> 2, sub = t & 3u;
+        const uint32_t row = u / static_cast<uint32_t>(p.groups);
+        const uint32_t cg = u - row * static_cast<uint32_t>(p.groups);
+        const int blk = static_cast<int>(cg * 4u + sub);
+        uint32_t sbyte = 0;
+        if (t < total && row < static_cast<uint32_t>(p.rows) && blk < nblk) {
+            float g;
+            const int s = seg_of(p.seg, row);
+            if (p.mode == 0)
+                g = global_scale_from_amax(p.amax_bits[s]);
+            else
+                g = p.g_in[s];
+            const uint4 *src = reinterpret_cast<const uint4 *>(p.X + static_cast<int64_t>(row) * p.ld + blk * 16);
+            const uint4 v0 = __ldg(src), v1 = __ldg(src + 1);
+            const uint32_t bmax = hmax16(vmax_mag(vmax_mag(0u, v0), v1));
+            const float bamax = __uint_as_float(bmax << 16);
+            const float s32 = __fdiv_rn(__fdiv_rn(bamax, 6.0f), g);
+            sbyte = f32_to_e4m3_satfinite(s32);
+            const float d = __fmul_rn(e4m3_to_f32(sbyte), g);
+            const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+            uint32_t packed[2] = {0u, 0u};
+            if (d == 0.0f) {
+                // zero scale: every code is +-0 with the sign of its input
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const uint32_t lo = (w[i] >> 15) & 1u, hi = (w[i] >> 31) & 1u;
+                    packed[i >> 2] |= ((lo << 3) | (hi << 7)) << ((i & 3) * 8);
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const float y0 = __fdiv_rn(bf16_lo(w[i]), d);
+                    const float y1 = __fdiv_rn(bf16_hi(w[i]), d);
+                    packed[i >> 2] |= f32x2_to_e2m1x2(y0, y1) << ((i & 3) * 8);
+                }
+            }
+            uint2 *dst = reinterpret_cast<uint2 *>(p.codes + static_cast<int64_t>(row) * (p.K >> 1) + blk * 8);
+            *dst = make_uint2(packed[0], packed[1]);
+        }
+        // gather the four scale bytes of this group into lane (lane & ~3)
+        const int g0 = lane & ~3;
+        const uint32_t b0 = __shfl_sync(0xFFFFFFFFu, sbyte, g0);
+        const uint32_t b1 = __shfl_sync(0xFFFFFFFFu, sbyte, g0 + 1);
+        const uint32_t b2 = __shfl_sync(0xFFFFFFFFu, sbyte, g0 + 2);
+        const uint32_t b3 = __shfl_sync(0xFFFFFFFFu, sbyte, g0 + 3);
+        if (sub == 0 && t < total) {
+            const uint32_t word = b0 | (b1 << 8) | (b2 << 16) | (b3 << 24);
+            const uint64_t tile = static_cast<uint64_t>(row >> 7) * p.groups + cg;
+            const uint32_t rr = row & 127u;
+            *reinterpret_cast<uint32_t *>(p.sf + tile * 512 + (rr & 31u) * 16 + (rr >> 5) * 4) = word;
+        }
+    }
+}
+
+// --------------------------------------------------------------- SwiGLU
+
+// h[r, j] = bf16( silu(gate[r, j]) * up[r, j] ), silu(v) = v / (1 + exp(-v))
+// in fp32; gate_up is [rows, 2F] with leading dimension ld.  Also folds
+// max|h| into *amax_bits (zero on entry).
+__global__ void __launch_bounds__(256) swiglu_kernel(const uint16_t *__restrict__ GU, int64_t ld, int32_t rows,
+                                                     int32_t F, uint16_t *__restrict__ H,
+                                                     uint32_t *__restrict__ amax_bits)
+{
+    const uint32_t cpr = static_cast<uint32_t>(F) >> 3;
+    const uint32_t total = static_cast<uint32_t>(rows) * cpr;
+    uint32_t m = 0;
+    for (uint32_t t = blockIdx.x * blockDim.x + threadIdx.x; t < total; t += gridDim.x * blockDim.x) {
+        const uint32_t r = t / cpr, j = t - r * cpr;
+        const uint16_t *rowp = GU + static_cast<int64_t>(r) * ld;
+        const uint4 gv = __ldg(reinterpret_cast<const uint4 *>(rowp) + j);
+        const uint4 uv = __ldg(reinterpret_cast<const uint4 *>(rowp + F) + j);
+        const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
+        const uint32_t uw[4] = {uv.x, uv.y, uv.z, uv.w};
+        uint32_t hw[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            float h2[2];
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+                const float g = k ? bf16_hi(gw[i]) : bf16_lo(gw[i]);
+                const float u = k ? bf16_hi(uw[i]) : bf16_lo(uw[i]);
+                const float sg = __fdiv_rn(g, __fadd_rn(1.0f, expf(-g)));
+                h2[k] = __fmul_rn(sg, u);
+            }
+            const __nv_bfloat162 b = __floats2bfloat162_rn(h2[0], h2[1]);
+            hw[i] = *reinterpret_cast<const uint32_t *>(&b);
+            m = vmax_mag(m, hw[i]);
+        }
+        reinterpret_cast<uint4 *>(H + static_cast<int64_t>(r) * F)[j] = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+    }
+    uint32_t v = hmax16(m);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+        v = max(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
+    __shared__ uint32_t s_max;
+    if (threadIdx.x == 0)
+        s_max = 0;
+    __syncthreads();
+    if ((threadIdx.x & 31) == 0)
+        atomicMax(&s_max, v);
+    __syncthreads();
+    if (threadIdx.x == 0 && s_max != 0)
+        atomicMax(amax_bits, s_max);
+}
+
+}  // namespace nvfp4

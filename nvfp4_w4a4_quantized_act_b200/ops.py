@@ -1,0 +1,278 @@
+"""ctypes binding of libnvfp4.so (declared in include/nvfp4.h).
+
+Argument marshalling only: every step of the quantize / GEMM path runs in the
+library's CUDA kernels.  torch supplies device memory (output and workspace
+allocation) and the current CUDA stream.  There is no CPU fallback: if the
+library is missing or the device is not an sm_100 GPU, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libnvfp4.so")
+
+NVFP4_STATIC_SCALE = 1
+NVFP4_OUT_FP32 = 2
+MAX_SEGMENTS = 16
+
+STATUS_NAMES = {
+    0: "NVFP4_OK", 1: "NVFP4_ERR_INVALID_ARG", 2: "NVFP4_ERR_UNSUPPORTED_SHAPE", 3: "NVFP4_ERR_MISALIGNED",
+    4: "NVFP4_ERR_CUDA", 5: "NVFP4_ERR_TIMEOUT", 6: "NVFP4_ERR_NONFINITE", 7: "NVFP4_ERR_WORKSPACE",
+    8: "NVFP4_ERR_NO_DEVICE",
+}
+
+EXPORTED = [
+    "nvfp4_sf_bytes", "nvfp4_quant_workspace_bytes", "nvfp4_workspace_bytes", "nvfp4_linear_act_scale_offset",
+    "nvfp4_quantize_weights", "nvfp4_quantize_act", "nvfp4_gemm_prequant", "nvfp4_linear_fused",
+    "nvfp4_linear", "nvfp4_swiglu_quantize", "nvfp4_get_status", "nvfp4_status_string",
+    "nvfp4_device_supported", "nvfp4_launch_count",
+]
+
+
+class Nvfp4Error(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {STATUS_NAMES.get(code, code)} ({status_string(code)})")
+
+
+class Segment(ctypes.Structure):
+    _fields_ = [("n_begin", ctypes.c_int64), ("n_end", ctypes.c_int64)]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libnvfp4.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is missing: build it with nvfp4_w4a4_quantized_act_b200.build.build()")
+    L = ctypes.CDLL(LIB_PATH)
+    i64, sz, vp, u8p, fp = ctypes.c_int64, ctypes.c_size_t, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p
+    segp = ctypes.POINTER(Segment)
+    sig = {
+        "nvfp4_sf_bytes": (sz, [i64, i64]),
+        "nvfp4_quant_workspace_bytes": (sz, [ctypes.c_int]),
+        "nvfp4_workspace_bytes": (sz, [i64, i64, i64, ctypes.c_int]),
+        "nvfp4_linear_act_scale_offset": (sz, []),
+        "nvfp4_quantize_weights": (ctypes.c_int, [vp, i64, i64, i64, segp, ctypes.c_int, u8p, u8p, fp, vp, sz, vp]),
+        "nvfp4_quantize_act": (ctypes.c_int, [vp, i64, i64, i64, u8p, u8p, fp, ctypes.c_uint, vp, sz, vp]),
+        "nvfp4_gemm_prequant": (ctypes.c_int, [u8p, u8p, fp, i64, i64, u8p, u8p, i64, segp, fp, ctypes.c_int, vp,
+                                               ctypes.c_uint, vp]),
+        "nvfp4_linear_fused": (ctypes.c_int, [vp, i64, i64, u8p, u8p, i64, segp, fp, ctypes.c_int, vp,
+                                              ctypes.c_uint, vp, sz, vp]),
+        "nvfp4_linear": (ctypes.c_int, [vp, i64, i64, u8p, u8p, fp, i64, vp, ctypes.c_uint, vp, sz, vp]),
+        "nvfp4_swiglu_quantize": (ctypes.c_int, [vp, i64, i64, i64, vp, u8p, u8p, fp, vp, sz, vp]),
+        "nvfp4_get_status": (ctypes.c_int, [vp]),
+        "nvfp4_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+        "nvfp4_device_supported": (ctypes.c_int, []),
+        "nvfp4_launch_count": (ctypes.c_uint64, []),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(L, name)
+        f.restype = res
+        f.argtypes = args
+    _lib = L
+    return L
+
+
+def status_string(code: int) -> str:
+    return lib().nvfp4_status_string(int(code)).decode()
+
+
+def _check(rc: int, where: str):
+    if rc != 0:
+        raise Nvfp4Error(rc, where)
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _p(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _segs(segments):
+    arr = (Segment * len(segments))(*[Segment(int(a), int(b)) for a, b in segments])
+    return arr, len(segments)
+
+
+def _require_cuda(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("nvfp4 ops take CUDA tensors only (there is no CPU path)")
+
+
+def device_supported() -> bool:
+    return bool(lib().nvfp4_device_supported())
+
+
+def launch_count() -> int:
+    return int(lib().nvfp4_launch_count())
+
+
+def get_status(stream=None) -> int:
+    """Synchronize the stream and return/clear the device status word."""
+    return int(lib().nvfp4_get_status(_stream(stream)))
+
+
+def sf_bytes(rows: int, K: int) -> int:
+    return int(lib().nvfp4_sf_bytes(rows, K))
+
+
+def quant_workspace_bytes(nseg: int = 1) -> int:
+    return int(lib().nvfp4_quant_workspace_bytes(nseg))
+
+
+def workspace_bytes(M: int, N: int, K: int, nseg: int = 1) -> int:
+    return int(lib().nvfp4_workspace_bytes(M, N, K, nseg))
+
+
+def act_scale_offset() -> int:
+    return int(lib().nvfp4_linear_act_scale_offset())
+
+
+def _empty_u8(n, device):
+    return torch.empty(max(int(n), 1), dtype=torch.uint8, device=device)
+
+
+@dataclass
+class QuantizedWeight:
+    """A (possibly fused) NVFP4 weight: codes [N, K/2], swizzled scales,
+    one FP32 global scale per module segment."""
+    codes: torch.Tensor
+    sf: torch.Tensor
+    g_w: torch.Tensor
+    segments: list
+    N: int
+    K: int
+
+
+def quantize_weights(W: torch.Tensor, segments=None, stream=None) -> QuantizedWeight:
+    """nvfp4_quantize_weights: per-module dynamic scales over row segments."""
+    _require_cuda(W)
+    assert W.dtype == torch.bfloat16 and W.dim() == 2 and W.stride(1) == 1
+    N, K = W.shape
+    segments = [(0, N)] if segments is None else [(int(a), int(b)) for a, b in segments]
+    dev = W.device
+    codes = _empty_u8(N * K // 2, dev)
+    sf = _empty_u8(sf_bytes(N, K), dev)
+    g_w = torch.empty(len(segments), dtype=torch.float32, device=dev)
+    ws = _empty_u8(quant_workspace_bytes(len(segments)), dev)
+    arr, n = _segs(segments)
+    _check(lib().nvfp4_quantize_weights(_p(W), N, K, W.stride(0), arr, n, _p(codes), _p(sf), _p(g_w), _p(ws),
+                                        ws.numel(), _stream(stream)), "nvfp4_quantize_weights")
+    return QuantizedWeight(codes[: N * K // 2].view(N, K // 2), sf, g_w, segments, N, K)
+
+
+def quantize_act(X: torch.Tensor, g_a: torch.Tensor | None = None, static_scale: bool = False, codes=None,
+                 sf=None, ws=None, stream=None):
+    """nvfp4_quantize_act -> (codes [M, K/2] u8, swizzled sf u8, g_a fp32[1])."""
+    _require_cuda(X)
+    assert X.dtype == torch.bfloat16 and X.dim() == 2 and X.stride(1) == 1
+    M, K = X.shape
+    dev = X.device
+    if codes is None:
+        codes = _empty_u8(M * K // 2, dev)
+    if sf is None:
+        sf = _empty_u8(sf_bytes(M, K), dev)
+    if g_a is None:
+        assert not static_scale
+        g_a = torch.empty(1, dtype=torch.float32, device=dev)
+    if ws is None:
+        ws = _empty_u8(quant_workspace_bytes(1), dev)
+    flags = NVFP4_STATIC_SCALE if static_scale else 0
+    _check(lib().nvfp4_quantize_act(_p(X), M, K, X.stride(0), _p(codes), _p(sf), _p(g_a), flags, _p(ws),
+                                    ws.numel(), _stream(stream)), "nvfp4_quantize_act")
+    return codes[: M * K // 2].view(M, K // 2), sf, g_a
+
+
+def gemm_prequant(a_codes, a_sf, g_a, M: int, K: int, w: QuantizedWeight, out=None, out_fp32=False, stream=None):
+    """nvfp4_gemm_prequant on already-quantized activations."""
+    _require_cuda(a_codes, a_sf, g_a)
+    dt = torch.float32 if out_fp32 else torch.bfloat16
+    if out is None:
+        out = torch.empty((M, w.N), dtype=dt, device=a_codes.device)
+    arr, n = _segs(w.segments)
+    flags = NVFP4_OUT_FP32 if out_fp32 else 0
+    _check(lib().nvfp4_gemm_prequant(_p(a_codes), _p(a_sf), _p(g_a), M, K, _p(w.codes), _p(w.sf), w.N, arr,
+                                     _p(w.g_w), n, _p(out), flags, _stream(stream)), "nvfp4_gemm_prequant")
+    return out
+
+
+def linear_fused(X: torch.Tensor, w: QuantizedWeight, out=None, out_fp32=False, ws=None, static_scale=False,
+                 stream=None):
+    """nvfp4_linear_fused: quantize X on the fly, fused-module GEMM with one
+    global scale per module segment."""
+    _require_cuda(X)
+    assert X.dtype == torch.bfloat16 and X.is_contiguous()
+    M, K = X.shape
+    assert K == w.K
+    dt = torch.float32 if out_fp32 else torch.bfloat16
+    if out is None:
+        out = torch.empty((M, w.N), dtype=dt, device=X.device)
+    if ws is None:
+        ws = _empty_u8(workspace_bytes(M, w.N, K, len(w.segments)), X.device)
+    arr, n = _segs(w.segments)
+    flags = (NVFP4_OUT_FP32 if out_fp32 else 0) | (NVFP4_STATIC_SCALE if static_scale else 0)
+    _check(lib().nvfp4_linear_fused(_p(X), M, K, _p(w.codes), _p(w.sf), w.N, arr, _p(w.g_w), n, _p(out), flags,
+                                    _p(ws), ws.numel(), _stream(stream)), "nvfp4_linear_fused")
+    return out
+
+
+def linear(X: torch.Tensor, w: QuantizedWeight, out=None, out_fp32=False, ws=None, stream=None):
+    """nvfp4_linear: single-module linear (uses g_w[0])."""
+    _require_cuda(X)
+    assert X.dtype == torch.bfloat16 and X.is_contiguous()
+    M, K = X.shape
+    dt = torch.float32 if out_fp32 else torch.bfloat16
+    if out is None:
+        out = torch.empty((M, w.N), dtype=dt, device=X.device)
+    if ws is None:
+        ws = _empty_u8(workspace_bytes(M, w.N, K, 1), X.device)
+    flags = NVFP4_OUT_FP32 if out_fp32 else 0
+    _check(lib().nvfp4_linear(_p(X), M, K, _p(w.codes), _p(w.sf), _p(w.g_w), w.N, _p(out), flags, _p(ws),
+                              ws.numel(), _stream(stream)), "nvfp4_linear")
+    return out
+
+
+def linear_workspace_views(ws: torch.Tensor, M: int, K: int):
+    """The activation scale, codes and scale factors a linear call left in
+    its workspace (for tests): (g_a fp32[1], codes [M, K/2], sf)."""
+    off = act_scale_offset()
+    g_a = ws[off: off + 4].view(torch.float32)
+    codes = ws[1024: 1024 + M * K // 2].view(M, K // 2)
+    sf_off = (1024 + M * K // 2 + 1023) // 1024 * 1024
+    sf = ws[sf_off: sf_off + sf_bytes(M, K)]
+    return g_a, codes, sf
+
+
+def swiglu_quantize(gate_up: torch.Tensor, h=None, codes=None, sf=None, g_h=None, ws=None, stream=None):
+    """nvfp4_swiglu_quantize -> (h bf16 [M, F], codes, sf, g_h)."""
+    _require_cuda(gate_up)
+    assert gate_up.dtype == torch.bfloat16 and gate_up.stride(1) == 1
+    M, F2 = gate_up.shape
+    F = F2 // 2
+    dev = gate_up.device
+    if h is None:
+        h = torch.empty((M, F), dtype=torch.bfloat16, device=dev)
+    if codes is None:
+        codes = _empty_u8(M * F // 2, dev)
+    if sf is None:
+        sf = _empty_u8(sf_bytes(M, F), dev)
+    if g_h is None:
+        g_h = torch.empty(1, dtype=torch.float32, device=dev)
+    if ws is None:
+        ws = _empty_u8(quant_workspace_bytes(1), dev)
+    _check(lib().nvfp4_swiglu_quantize(_p(gate_up), M, F, gate_up.stride(0), _p(h), _p(codes), _p(sf), _p(g_h),
+                                       _p(ws), ws.numel(), _stream(stream)), "nvfp4_swiglu_quantize")
+    return h, codes[: M * F // 2].view(M, F // 2), sf, g_h

@@ -1,0 +1,88 @@
+"""The C ABI library builds, loads and exports every symbol the header
+declares; host-side argument checks return their status codes before any
+CUDA work (these calls need no GPU)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from nvfp4_w4a4_quantized_act_b200 import build as nbuild
+from nvfp4_w4a4_quantized_act_b200 import ops
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "nvfp4.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    nbuild.build()
+    return ops.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(nvfp4_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declarations_are_exported(L):
+    names = declared_functions()
+    assert len(names) >= 14
+    for n in names:
+        assert hasattr(L, n), n
+    assert sorted(ops.EXPORTED) == names
+
+
+def test_sizes(L):
+    assert ops.sf_bytes(8192, 5120) == 8192 * 320
+    assert ops.sf_bytes(64, 256) == 128 * 16
+    assert ops.sf_bytes(1, 16) == 128 * 4
+    assert ops.sf_bytes(5, 17) == 0
+    assert ops.quant_workspace_bytes(1) >= 4 and ops.quant_workspace_bytes(0) == 0
+    ws = ops.workspace_bytes(8192, 34816, 5120, 2)
+    assert ws >= 8192 * 5120 // 2 + 8192 * 320 + 1024
+    assert ops.act_scale_offset() == 256
+
+
+def _segarr(pairs):
+    return (ops.Segment * len(pairs))(*[ops.Segment(a, b) for a, b in pairs])
+
+
+def test_argument_errors_return_before_launch(L):
+    i64 = ctypes.c_int64
+    fake = ctypes.c_void_p(1 << 20)  # 16-byte aligned, never dereferenced: checks fail first
+    mis = ctypes.c_void_p((1 << 20) + 8)
+    # null input
+    assert L.nvfp4_quantize_act(None, 8, 64, 64, fake, fake, fake, 0, fake, 256, None) == 1
+    # K not a multiple of 16
+    assert L.nvfp4_quantize_act(fake, 8, 40, 40, fake, fake, fake, 0, fake, 256, None) == 2
+    # leading dimension smaller than K
+    assert L.nvfp4_quantize_act(fake, 8, 64, 32, fake, fake, fake, 0, fake, 256, None) == 1
+    # misaligned input
+    assert L.nvfp4_quantize_act(mis, 8, 64, 64, fake, fake, fake, 0, fake, 256, None) == 3
+    # unknown flag bit
+    assert L.nvfp4_quantize_act(fake, 8, 64, 64, fake, fake, fake, 1 << 7, fake, 256, None) == 1
+    # workspace too small
+    assert L.nvfp4_quantize_act(fake, 8, 64, 64, fake, fake, fake, 0, fake, 2, None) == 7
+    segs_ok = _segarr([(0, 10), (10, 32)])
+    # GEMM: K % 64
+    assert L.nvfp4_gemm_prequant(fake, fake, fake, 8, 96, fake, fake, 32, segs_ok, fake, 2, fake, 0, None) == 2
+    # segments not covering [0, N)
+    bad = _segarr([(0, 10), (12, 32)])
+    assert L.nvfp4_gemm_prequant(fake, fake, fake, 8, 128, fake, fake, 32, bad, fake, 2, fake, 0, None) == 1
+    short = _segarr([(0, 10), (10, 30)])
+    assert L.nvfp4_gemm_prequant(fake, fake, fake, 8, 128, fake, fake, 32, short, fake, 2, fake, 0, None) == 1
+    # too many segments
+    many = _segarr([(i, i + 1) for i in range(17)])
+    assert L.nvfp4_gemm_prequant(fake, fake, fake, 8, 128, fake, fake, 17, many, fake, 17, fake, 0, None) == 1
+    # negative sizes
+    assert L.nvfp4_gemm_prequant(fake, fake, fake, -1, 128, fake, fake, 32, segs_ok, fake, 2, fake, 0, None) == 1
+    # linear_fused: workspace too small
+    assert L.nvfp4_linear_fused(fake, 8, 128, fake, fake, 32, segs_ok, fake, 2, fake, 0, fake, 16, None) == 7
+    # weights: misaligned leading dimension
+    assert L.nvfp4_quantize_weights(fake, 32, 64, 68, segs_ok, 2, fake, fake, fake, fake, 256, None) == 3
+    # SwiGLU: F % 16
+    assert L.nvfp4_swiglu_quantize(fake, 8, 24, 48, fake, fake, fake, fake, fake, 256, None) == 2
+    for code in range(9):
+        assert ops.status_string(code)
