@@ -1,0 +1,501 @@
+"""Benchmark of the NVFP4 W4A4 linear path on B200.
+
+Workload (default): the full stack of 496 linear layers of a 48 Gated-DeltaNet
+/ 16 attention hybrid at hidden size 5120, run on one 8192-token prefill
+chunk.  Every input-sharing group of modules is one fused GEMM with a global
+scale per module (4 GEMMs a layer, 256 a step):
+
+  GDN layer       in_proj [qkv 8192 | z 6144 | b 48 | a 48] <- X (5120)
+                  out      5120 <- Y (6144)
+                  gate_up [gate 17408 | up 17408] <- X2 (5120)
+                  down     5120 <- h = silu(gate) * up (17408)
+  attention layer qkv [q+gate 12288 | k 1024 | v 1024] <- X, o 5120 <- Y,
+                  gate_up, down as above
+
+A step quantizes every GEMM input on the fly (per-tensor dynamic global
+scale), runs the block-scaled FP4 GEMMs with the per-module global-scale
+epilogue, and computes + quantizes the MLP intermediate.  Weights are random
+N(0, 0.02), quantized once offline (per module).  Activations X, X2 ~ N(0,1)
+with 4 outlier channels x50, Y ~ N(0,1); all synthetic and seeded.
+
+Prints one JSON line (rank 0).  `--impl reference` times the CPU oracle on a
+bounded sample of the same workload instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+TOKENS = 8192
+HIDDEN = 5120
+METRIC = "NVFP4 W4A4 linear TFLOPS (quant+GEMM) at prefill shapes; % of FP4 & HBM peak"
+WORKLOAD = "496-linear hybrid stack (48 GDN + 16 attention layers, hidden 5120, MLP 17408), one 8192-token prefill chunk"
+FP4_PER_BF16 = 4.0  # dense FP4 : dense BF16 tensor throughput on B200 (9 : 2.25 PFLOP/s nominal)
+FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["nvfp4", "reference"], default="nvfp4")
+    ap.add_argument("--layers", type=int, default=64, help="layers in the stack (64 = the full model)")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    return ap.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK), "fallback"
+
+
+# --------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling while the timed region runs."""
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.file = None
+
+    def start(self):
+        try:
+            self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=self.file, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        out = {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        if self.proc is None:
+            return out
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.file.flush()
+        self.file.seek(0)
+        rows = [r.split(",") for r in self.file.read().strip().splitlines() if r.strip()]
+        self.file.close()
+        os.unlink(self.file.name)
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        sm, mx, reasons = [], [], set()
+        for r in rows:
+            try:
+                sm.append(float(r[1]))
+                mx.append(float(r[2]))
+                for n, v in zip(names, r[5:9]):
+                    if v.strip().lower() == "active":
+                        reasons.add(n)
+            except (ValueError, IndexError):
+                pass
+        if sm:
+            out["sm_mhz"] = statistics.median(sm)
+            out["sm_max_mhz"] = max(mx)
+        out["reasons"] = sorted(reasons)
+        out["samples"] = len(sm)
+        return out
+
+
+# ------------------------------------------------------------ the stack
+
+def stack_flops(layers) -> float:
+    f = 0.0
+    for _, lins in layers:
+        for lin in lins:
+            f += 2.0 * TOKENS * lin.N * lin.K
+    return f
+
+
+class Stack:
+    """Quantized weights of the stack plus the reusable activation/output
+    buffers of one prefill chunk."""
+
+    def __init__(self, n_layers: int, device, seed: int = 1000):
+        from nvfp4_w4a4_quantized_act_b200 import ops
+        from nvfp4_w4a4_quantized_act_b200 import workloads as wl
+        self.ops = ops
+        self.layers = wl.stack_layers()[:n_layers]
+        self.weights = []  # per layer: 4 QuantizedWeight
+        for li, (kind, lins) in enumerate(self.layers):
+            qs = []
+            for gi, lin in enumerate(lins):
+                parts = [wl.weight_normal_cuda(m.width, lin.K, m.sigma, seed + 97 * li + 11 * gi + j, device)
+                         for j, m in enumerate(lin.modules)]
+                W = torch.cat(parts, 0) if len(parts) > 1 else parts[0]
+                del parts
+                qs.append(ops.quantize_weights(W, lin.segments))
+                del W
+            self.weights.append(qs)
+        torch.cuda.synchronize()
+        # activations (synthetic, seeded) and buffers
+        self.X = wl.activation_normal_cuda(TOKENS, HIDDEN, 11, device=device)
+        self.X2 = wl.activation_normal_cuda(TOKENS, HIDDEN, 12, device=device)
+        self.Y = wl.activation_normal_cuda(TOKENS, 6144, 13, n_outliers=0, device=device)
+        self.outs = {}
+        for _, lins in self.layers[:4]:
+            for lin in lins:
+                self.outs.setdefault((lin.name, lin.N), torch.empty((TOKENS, lin.N), dtype=torch.bfloat16,
+                                                                     device=device))
+        maxK = max(lin.K for _, lins in self.layers for lin in lins)
+        self.a_codes = torch.empty(TOKENS * maxK // 2, dtype=torch.uint8, device=device)
+        self.a_sf = torch.empty(ops.sf_bytes(TOKENS, maxK), dtype=torch.uint8, device=device)
+        self.g_a = torch.empty(1, dtype=torch.float32, device=device)
+        self.qws = torch.empty(ops.quant_workspace_bytes(1), dtype=torch.uint8, device=device)
+        self.h = torch.empty((TOKENS, 17408), dtype=torch.bfloat16, device=device)
+        self.lin_ws = torch.empty(ops.workspace_bytes(TOKENS, 0, maxK), dtype=torch.uint8, device=device)
+        self.flops = stack_flops(self.layers)
+        self.gemm_flops = [2.0 * TOKENS * lin.N * lin.K for _, lins in self.layers for lin in lins]
+
+    def _input(self, lin):
+        if lin.name in ("gdn_out", "attn_o"):
+            return self.Y
+        if lin.name == "gate_up":
+            return self.X2
+        return self.X
+
+    def step_split(self, gemm_events=None):
+        """One step through nvfp4_quantize_act / nvfp4_swiglu_quantize /
+        nvfp4_gemm_prequant, with CUDA events around each GEMM launch."""
+        ops = self.ops
+        k = 0
+        for qs, (_, lins) in zip(self.weights, self.layers):
+            for lin, qw in zip(lins, qs):
+                out = self.outs[(lin.name, lin.N)]
+                if lin.name == "down":
+                    gu = self.outs[("gate_up", 34816)]
+                    _, hc, hsf, gh = ops.swiglu_quantize(gu, h=self.h, codes=self.a_codes, sf=self.a_sf,
+                                                         g_h=self.g_a, ws=self.qws)
+                    ac, asf = hc, hsf
+                else:
+                    ac, asf, _ = ops.quantize_act(self._input(lin), g_a=self.g_a, codes=self.a_codes, sf=self.a_sf,
+                                                  ws=self.qws)
+                if gemm_events is not None:
+                    gemm_events[k][0].record()
+                ops.gemm_prequant(ac, asf, self.g_a, TOKENS, lin.K, qw, out=out)
+                if gemm_events is not None:
+                    gemm_events[k][1].record()
+                k += 1
+
+    def step_public(self):
+        """One step through the user-facing calls (nvfp4_linear_fused for
+        every fused GEMM, nvfp4_swiglu_quantize + nvfp4_gemm_prequant for the
+        down projection)."""
+        ops = self.ops
+        last = None
+        for qs, (_, lins) in zip(self.weights, self.layers):
+            for lin, qw in zip(lins, qs):
+                out = self.outs[(lin.name, lin.N)]
+                if lin.name == "down":
+                    gu = self.outs[("gate_up", 34816)]
+                    _, hc, hsf, gh = ops.swiglu_quantize(gu, h=self.h, codes=self.a_codes, sf=self.a_sf,
+                                                         g_h=self.g_a, ws=self.qws)
+                    ops.gemm_prequant(hc, hsf, gh, TOKENS, lin.K, qw, out=out)
+                else:
+                    ops.linear_fused(self._input(lin), qw, out=out, ws=self.lin_ws)
+                last = out
+        return last
+
+
+# -------------------------------------------------------------- GPU arm
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import torch.distributed as dist
+        import datetime
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda" if torch.cuda.is_available() else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def bench_gpu(args, rank, world, local):
+    from nvfp4_w4a4_quantized_act_b200 import build as nbuild
+    from nvfp4_w4a4_quantized_act_b200 import ops
+    nbuild.build()
+    if not ops.device_supported():
+        raise RuntimeError("the current device is not an sm_100 GPU")
+    dev = f"cuda:{local}"
+    stack = Stack(args.layers, dev)
+    n_gemm = len(stack.gemm_flops)
+    stream = torch.cuda.current_stream()
+
+    for _ in range(args.warmup):
+        stack.step_split()
+    torch.cuda.synchronize()
+    if ops.get_status() != 0:
+        raise RuntimeError("device status set during warm-up")
+
+    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_gemm)]
+          for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    l0 = ops.launch_count()
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for s in range(args.steps):
+        stack.step_split(ev[s])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    launches = ops.launch_count() - l0
+    elapsed_ms = max_over_ranks(t_start.elapsed_time(t_end), world)
+    gemm_ms = [sum(ev[s][k][0].elapsed_time(ev[s][k][1]) for s in range(args.steps)) / args.steps
+               for k in range(n_gemm)]
+    status = ops.get_status()
+    if status != 0:
+        raise RuntimeError(f"device status {status} after the timed region")
+
+    ms_per_step = elapsed_ms / args.steps
+    value = stack.flops * world / (ms_per_step * 1e-3) / 1e12
+    gemm_tflops = sum(stack.gemm_flops) / (sum(gemm_ms) * 1e-3) / 1e12
+    pk, pk_kind = peaks()
+    fp4_peak = pk["bf16_tflops_sustained"] * FP4_PER_BF16
+
+    # quantize kernel throughput: one activation [8192, 5120] at HBM roofline
+    quant = quantize_roofline(stack, pk, pk_kind)
+
+    e2e = None
+    if not args.no_e2e:
+        e2e = bench_e2e(stack, args, world)
+
+    res = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "TFLOPS",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_per_step, 3),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "nvfp4 (e2m1 + e4m3 block scales) x nvfp4 -> fp32 accumulate -> bf16",
+        "data": "synthetic (seeded N(0,1) activations with outlier channels; random N(0,0.02) weights)",
+        "config": {
+            "workload": WORKLOAD if args.layers == 64 else f"{args.layers}-layer prefix of the stack",
+            "tokens": TOKENS, "hidden": HIDDEN, "layers": args.layers, "gemms_per_step": n_gemm,
+            "linears_per_step": sum(len(m.modules) for _, lins in stack.layers for m in lins),
+            "gemm_tflop_per_step": round(stack.flops / 1e12, 2),
+            "l2": "no flush: each step streams 13.4 GB of NVFP4 weights, far larger than the 126 MB L2",
+            "parallelism": f"replicas x{world} (no collectives)",
+        },
+        "roofline": {
+            "kernel": "gemm_nvf4_kernel (tcgen05 block-scaled FP4 GEMM + per-module scale epilogue)",
+            "bound": "tensor",
+            "achieved": round(gemm_tflops, 1),
+            "peak": round(fp4_peak, 1),
+            "unit": "TFLOP/s",
+            "frac": round(gemm_tflops / fp4_peak, 4),
+            "traffic": None,
+            "peak_basis": f"{pk_kind} bf16 sustained {pk['bf16_tflops_sustained']} TF/s x {FP4_PER_BF16} "
+                          "(nominal dense FP4:BF16 ratio)",
+            "frac_of_datasheet_9pf": round(gemm_tflops / 9000.0, 4),
+        },
+        "quantize_roofline": quant,
+        "gemm_share_of_step": round(sum(gemm_ms) / ms_per_step, 4),
+        "gpu_launches": int(launches),
+        "clocks": clk,
+    }
+    if e2e is not None:
+        res["e2e"] = e2e
+    return res
+
+
+def quantize_roofline(stack, pk, pk_kind):
+    from nvfp4_w4a4_quantized_act_b200 import ops
+    X = stack.X
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=X.device)
+    ts = []
+    for i in range(13):
+        flush.zero_()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        ops.quantize_act(X, g_a=stack.g_a, codes=stack.a_codes, sf=stack.a_sf, ws=stack.qws)
+        e.record()
+        e.synchronize()
+        if i >= 3:
+            ts.append(s.elapsed_time(e))
+    ms = statistics.median(ts)
+    alg = TOKENS * HIDDEN * (2 + 0.5 + 1 / 16)
+    gbs = alg / (ms * 1e-3) / 1e9
+    return {"kernel": "amax_kernel + quantize_kernel (dynamic per-tensor scale), X [8192, 5120] bf16",
+            "bound": "hbm", "achieved": round(gbs, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
+            "frac": round(gbs / pk["hbm_gbs"], 4), "us": round(ms * 1e3, 2),
+            "algorithmic_bytes": int(alg), "peak_basis": pk_kind, "l2": "256 MB flush before each launch"}
+
+
+def bench_e2e(stack, args, world):
+    """Same workload through the user-facing calls, with this step's inputs
+    copied from pinned host memory and the final output read back."""
+    hX = stack.X.cpu().pin_memory()
+    hX2 = stack.X2.cpu().pin_memory()
+    hY = stack.Y.cpu().pin_memory()
+    last_shape = stack.outs[("down", HIDDEN)].shape
+    hOut = torch.empty(last_shape, dtype=torch.bfloat16).pin_memory()
+    h2d = hX.numel() * 2 + hX2.numel() * 2 + hY.numel() * 2
+    d2h = hOut.numel() * 2
+
+    def step():
+        stack.X.copy_(hX, non_blocking=True)
+        stack.X2.copy_(hX2, non_blocking=True)
+        stack.Y.copy_(hY, non_blocking=True)
+        last = stack.step_public()
+        hOut.copy_(last, non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(args.steps):
+        step()
+    e.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = max_over_ranks(s.elapsed_time(e), world) / args.steps
+    return {"value": round(stack.flops * world / (ms * 1e-3) / 1e12, 2), "unit": "TFLOPS",
+            "ms_per_step": round(ms, 3), "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+            "api": "nvfp4_linear_fused / nvfp4_swiglu_quantize / nvfp4_gemm_prequant"}
+
+
+# ------------------------------------------------------ CPU oracle legs
+
+def oracle_sample_time(seconds: float, seed: int = 0):
+    """Time the oracle on a bounded sample of the stack: quantize the rows it
+    needs of one activation and one gate_up weight, then compute sampled
+    outputs of that GEMM by fp64 dot products, until `seconds` pass.
+    Returns (flops, seconds, outputs)."""
+    import oracle
+    from nvfp4_w4a4_quantized_act_b200 import workloads as wl
+    rng = np.random.default_rng(seed)
+    K = HIDDEN
+    rows = 64
+    x = wl.activation_normal(rows, K, 11)
+    w = wl.weight_normal(256, K, 0.02, 1000)
+    xb, wb = wl.bf16_bits(x), wl.bf16_bits(w)
+    flops = 0.0
+    outs = 0
+    t0 = time.perf_counter()
+    while True:
+        ca, sa, ga = oracle.quantize_tensor(xb)
+        cw, sw, gw = oracle.quantize_tensor(wb)
+        ms = rng.integers(0, rows, 1024)
+        ns = rng.integers(0, wb.shape[0], 1024)
+        oracle.linear_sampled(ca, sa, ga, cw, sw, gw, ms, ns)
+        flops += 2.0 * K * len(ms)
+        outs += len(ms)
+        el = time.perf_counter() - t0
+        if el >= seconds:
+            return flops, el, outs
+
+
+def cpu_baseline(seconds: float):
+    flops, el, outs = oracle_sample_time(seconds)
+    return {"value": flops / el / 1e12, "unit": "TFLOPS", "cores": 1, "kind": "oracle",
+            "sample": f"{outs} outputs of a [8192,5120]x[34816,5120]^T gate_up GEMM (K=5120) with on-the-fly "
+                      f"quantization of the 64 activation rows and 256 weight rows they use, repeated for "
+                      f"{el:.1f} s; single-threaded C oracle, fp64 dot products"}
+
+
+def bench_reference(args, rank, world):
+    if rank != 0:
+        return None
+    per_step = max(2.0, min(20.0, 60.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        oracle_sample_time(per_step / 4)
+    tot_f, tot_t = 0.0, 0.0
+    for _ in range(args.steps):
+        f, t, outs = oracle_sample_time(per_step)
+        tot_f += f
+        tot_t += t
+    v = tot_f / tot_t / 1e12
+    return {
+        "impl": "reference", "metric": METRIC, "value": v, "unit": "TFLOPS", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": tot_t / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64 (oracle GEMM)",
+        "data": "synthetic", "config": {"workload": WORKLOAD, "tokens": TOKENS, "hidden": HIDDEN},
+        "cpu_baseline": {"value": v, "unit": "TFLOPS", "cores": 1, "kind": "oracle",
+                         "sample": f"each step: {per_step:.1f} s of sampled gate_up outputs with quantization"},
+        "e2e": {"value": v, "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        # the oracle arm runs on rank 0's host cores only; other ranks exit at once
+        rank = int(os.environ.get("RANK", "0"))
+        res = bench_reference(args, rank, int(os.environ.get("WORLD_SIZE", "1")))
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+    rank, world, local = dist_setup(args)
+    try:
+        res = bench_gpu(args, rank, world, local)
+        if rank == 0 and res is not None and not args.no_cpu_baseline:
+            res["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
+        if rank == 0 and res is not None:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()
