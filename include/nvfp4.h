@@ -183,6 +183,42 @@ int nvfp4_device_supported(void);
  * this process, for launch accounting. */
 uint64_t nvfp4_launch_count(void);
 
+/* Allocation-free variant of nvfp4_linear_fused (no counterpart in the
+ * paper: this is a deployment convenience, not part of the method).
+ *
+ * Some callers cannot allocate device memory on the path that runs the
+ * layer: a runtime or plugin host that owns every device allocation and
+ * hands its operators no allocator, or a latency-critical serving loop in
+ * which cudaMalloc's implicit device-wide synchronization is not allowed.
+ * Such a caller cannot provide the scratch workspace that nvfp4_linear_fused
+ * needs for the quantized activation.  This entry point keeps that scratch in
+ * a fixed device array inside the library instead, and allocates nothing: it
+ * calls no cudaMalloc / cudaFree and no allocating library routine.
+ *
+ * Arguments are those of nvfp4_linear_fused without the workspace; the
+ * caller still passes X, the weight, the segment table and `out`.  Only the
+ * dynamic activation scale is supported (NVFP4_STATIC_SCALE is rejected with
+ * NVFP4_ERR_INVALID_ARG); NVFP4_OUT_FP32 is accepted.
+ *
+ * Limits: M*K <= NVFP4_NOALLOC_MAX_ELEMS and nvfp4_sf_bytes(M, K) <=
+ * NVFP4_NOALLOC_MAX_SF_BYTES (about 2.5 MB of device memory, which every GPU
+ * that loads the library keeps until the process exits).  Larger inputs are
+ * rejected with NVFP4_ERR_WORKSPACE before anything is launched.
+ *
+ * The first call on a device looks up the array's device address (once per
+ * device, with that device current); make that first call before any stream
+ * capture begins.  All calls share the one array and it keeps the last
+ * call's contents (the amax word is cleared by every call): calls that can
+ * overlap on the GPU -- on different streams without ordering, or from
+ * several host threads -- race with each other and must be serialized by the
+ * caller. */
+#define NVFP4_NOALLOC_MAX_ELEMS (1ll << 22)
+#define NVFP4_NOALLOC_MAX_SF_BYTES (1ll << 19)
+int nvfp4_linear_fused_noalloc(const void *X, int64_t M, int64_t K,
+                               const uint8_t *w_codes, const uint8_t *w_sf, int64_t N,
+                               const nvfp4_segment *segs, const float *g_w, int nseg,
+                               void *out, unsigned flags, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

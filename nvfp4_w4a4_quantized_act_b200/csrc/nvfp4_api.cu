@@ -520,3 +520,85 @@ int nvfp4_device_supported(void)
 uint64_t nvfp4_launch_count(void) { return g_launches.load(); }
 
 }  // extern "C"
+
+// ------------------------------------------------- allocation-free linear
+
+namespace {
+
+// Scratch of nvfp4_linear_fused_noalloc, laid out like a linear workspace:
+// [amax word | g_a | activation codes | activation scale factors].
+constexpr size_t kNoAllocCodesBytes = static_cast<size_t>(NVFP4_NOALLOC_MAX_ELEMS) / 2;
+constexpr size_t kNoAllocSfOff = kLinCodesOff + kNoAllocCodesBytes;
+constexpr size_t kNoAllocBytes = kNoAllocSfOff + static_cast<size_t>(NVFP4_NOALLOC_MAX_SF_BYTES);
+static_assert(kNoAllocSfOff % 1024 == 0, "scale factors must stay 16-byte aligned for the bulk copies");
+
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocBytes];
+
+// Device address of g_noalloc_scratch per device (the host-side symbol is a
+// stand-in, never a device pointer).
+uint8_t *g_noalloc_ptr[kMaxDevices] = {};
+std::mutex g_noalloc_mu;
+
+uint8_t *noalloc_scratch()
+{
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+        return nullptr;
+    if (g_noalloc_ptr[dev] != nullptr)
+        return g_noalloc_ptr[dev];
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (g_noalloc_ptr[dev] == nullptr) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
+            return nullptr;
+        g_noalloc_ptr[dev] = static_cast<uint8_t *>(p);
+    }
+    return g_noalloc_ptr[dev];
+}
+
+}  // namespace
+
+extern "C" int nvfp4_linear_fused_noalloc(const void *X, int64_t M, int64_t K, const uint8_t *w_codes,
+                                          const uint8_t *w_sf, int64_t N, const nvfp4_segment *segs,
+                                          const float *g_w, int nseg, void *out, unsigned flags, void *stream)
+{
+    if ((flags & ~static_cast<unsigned>(NVFP4_OUT_FP32)) != 0)
+        return NVFP4_ERR_INVALID_ARG;
+    int rc = check_gemm_shape(M, N, K);
+    if (rc != NVFP4_OK)
+        return rc;
+    nvfp4::SegRows seg;
+    rc = check_segments(segs, nseg, N, &seg);
+    if (rc != NVFP4_OK)
+        return rc;
+    if (M * K > NVFP4_NOALLOC_MAX_ELEMS || sf_bytes_i(M, K) > NVFP4_NOALLOC_MAX_SF_BYTES)
+        return NVFP4_ERR_WORKSPACE;
+    if (M == 0 || N == 0)
+        return NVFP4_OK;
+    if (X == nullptr || w_codes == nullptr || w_sf == nullptr || g_w == nullptr || out == nullptr)
+        return NVFP4_ERR_INVALID_ARG;
+    if (!aligned16(X) || K % 8 != 0 || !aligned16(w_codes) || !aligned16(w_sf) ||
+        (reinterpret_cast<uintptr_t>(g_w) & 3u) ||
+        (reinterpret_cast<uintptr_t>(out) & ((flags & NVFP4_OUT_FP32) ? 3u : 1u)))
+        return NVFP4_ERR_MISALIGNED;
+    DeviceState *d = device_state();
+    if (d == nullptr)
+        return NVFP4_ERR_CUDA;
+    if (!d->supported)
+        return NVFP4_ERR_NO_DEVICE;
+    uint8_t *base = noalloc_scratch();
+    if (base == nullptr)
+        return NVFP4_ERR_CUDA;
+    uint32_t *amax = reinterpret_cast<uint32_t *>(base);
+    float *g_a = reinterpret_cast<float *>(base + kLinScaleOff);
+    uint8_t *a_codes = base + kLinCodesOff;
+    uint8_t *a_sf = base + kNoAllocSfOff;
+    nvfp4::SegRows one_seg;
+    nvfp4_segment one = {0, M};
+    check_segments(&one, 1, M, &one_seg);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    rc = run_quantize(d, X, M, K, K, one_seg, a_codes, a_sf, g_a, g_a, true, amax, s);
+    if (rc != NVFP4_OK)
+        return rc;
+    return run_gemm(d, a_codes, a_sf, g_a, M, K, w_codes, w_sf, N, seg, g_w, out, flags, s);
+}

@@ -30,7 +30,7 @@ EXPORTED = [
     "nvfp4_sf_bytes", "nvfp4_quant_workspace_bytes", "nvfp4_workspace_bytes", "nvfp4_linear_act_scale_offset",
     "nvfp4_quantize_weights", "nvfp4_quantize_act", "nvfp4_gemm_prequant", "nvfp4_linear_fused",
     "nvfp4_linear", "nvfp4_swiglu_quantize", "nvfp4_get_status", "nvfp4_status_string",
-    "nvfp4_device_supported", "nvfp4_launch_count",
+    "nvfp4_device_supported", "nvfp4_launch_count", "nvfp4_linear_fused_noalloc",
 ]
 
 
@@ -74,6 +74,8 @@ def lib() -> ctypes.CDLL:
         "nvfp4_status_string": (ctypes.c_char_p, [ctypes.c_int]),
         "nvfp4_device_supported": (ctypes.c_int, []),
         "nvfp4_launch_count": (ctypes.c_uint64, []),
+        "nvfp4_linear_fused_noalloc": (ctypes.c_int, [vp, i64, i64, u8p, u8p, i64, segp, fp, ctypes.c_int, vp,
+                                                      ctypes.c_uint, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -276,3 +278,25 @@ def swiglu_quantize(gate_up: torch.Tensor, h=None, codes=None, sf=None, g_h=None
     _check(lib().nvfp4_swiglu_quantize(_p(gate_up), M, F, gate_up.stride(0), _p(h), _p(codes), _p(sf), _p(g_h),
                                        _p(ws), ws.numel(), _stream(stream)), "nvfp4_swiglu_quantize")
     return h, codes[: M * F // 2].view(M, F // 2), sf, g_h
+
+
+NOALLOC_MAX_ELEMS = 1 << 22
+NOALLOC_MAX_SF_BYTES = 1 << 19
+
+
+def linear_fused_noalloc(X: torch.Tensor, w: QuantizedWeight, out=None, out_fp32=False, stream=None):
+    """nvfp4_linear_fused_noalloc: the fused linear with its activation
+    scratch in the library's own fixed device array, for callers that cannot
+    allocate device memory where the layer runs (M*K <= 2^22).  `out` may be
+    passed to keep the call free of allocations on the Python side too."""
+    _require_cuda(X)
+    assert X.dtype == torch.bfloat16 and X.is_contiguous()
+    M, K = X.shape
+    dt = torch.float32 if out_fp32 else torch.bfloat16
+    if out is None:
+        out = torch.empty((M, w.N), dtype=dt, device=X.device)
+    arr, n = _segs(w.segments)
+    flags = NVFP4_OUT_FP32 if out_fp32 else 0
+    _check(lib().nvfp4_linear_fused_noalloc(_p(X), M, K, _p(w.codes), _p(w.sf), w.N, arr, _p(w.g_w), n, _p(out),
+                                            flags, _stream(stream)), "nvfp4_linear_fused_noalloc")
+    return out
