@@ -12,15 +12,20 @@
 // checkpoints are served by a kernel that fuses those modules into one GEMM
 // (same page, "The abstract" and "The deep dive").
 //
-// Structure (one CTA per SM, 6 warps):
-//   warp 0      TMA producer: codes tiles by 2-D tiled TMA (128-byte swizzle),
-//               scale-factor tiles by 1-D bulk copies, into a 4-stage ring.
-//   warp 1      allocates 512 TMEM columns; one lane issues tcgen05.cp for the
-//               scale factors and tcgen05.mma (kind::mxf4nvf4, 128x192x64 per
-//               instruction) and commits stage / accumulator barriers.
-//   warps 2..5  epilogue: tcgen05.ld of the fp32 accumulator, x alpha[n],
-//               bf16 (or fp32) stores.  Two accumulator buffers in TMEM let the
-//               epilogue of tile i overlap the main loop of tile i+1.
+// Tile 128 x 256 (x 256 of K per pipeline stage), one CTA per SM, 12 warps:
+//   warp 0      TMA producer: codes by 2-D tiled TMA (128-byte swizzle),
+//               scale-factor tiles by 1-D bulk copies, 4-stage ring.
+//   warp 1      allocates 512 TMEM columns; one lane issues the MMAs.  The
+//               256-column tile is two 128-column accumulators and the
+//               128x128x64 kind::mxf4nvf4 MMAs alternate between them:
+//               back-to-back MMAs into one accumulator wait on each other,
+//               two independent chains keep the tensor pipe full.
+//   warp 2      one lane copies each stage's scale factors shared -> TMEM
+//               (tcgen05.cp) into that stage's own TMEM buffer; copies issued
+//               from a warp other than the MMA warp overlap the MMAs.
+//   warps 4..11 epilogue: two warps per TMEM lane quarter, each drains 128
+//               accumulator columns into registers, releases TMEM (so the next
+//               tile's MMAs start), then applies alpha[n] and stores.
 // No load uses cluster multicast.  Every mbarrier wait is bounded in time;
 // when a wait runs out the kernel latches kStatusTimeout and unwinds.
 #pragma once
@@ -35,29 +40,33 @@
 namespace nvfp4 {
 namespace gemm {
 
-constexpr int BM = 128;            // rows of A per tile (TMEM lanes)
-constexpr int BN = 192;            // rows of W per tile (accumulator columns)
-constexpr int BK_BYTES = 128;      // 256 fp4 values of K per stage = one swizzle row
-constexpr int KB_PER_STAGE = 4;    // MMA K-steps (64 values) per stage
+constexpr int BM = 128;             // rows of A per tile (TMEM lanes)
+constexpr int BN = 256;             // rows of W per tile (accumulator columns)
+constexpr int HALF_N = 128;         // N of one MMA / one accumulator
+constexpr int BK_BYTES = 128;       // 256 fp4 values of K per stage = one swizzle row
+constexpr int KB_PER_STAGE = 4;     // MMA K-steps (64 values) per stage
 constexpr int STAGES = 4;
 constexpr uint32_t A_BYTES = BM * BK_BYTES;                 // 16 KB
-constexpr uint32_t B_BYTES = BN * BK_BYTES;                 // 24 KB
-constexpr uint32_t SFA_BYTES = KB_PER_STAGE * 512;          // one 128-row scale tile per K-step
-constexpr uint32_t SFB_BYTES = 2 * KB_PER_STAGE * 512;      // two 128-row scale tiles per K-step
-constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;  // 46 KB, 1024-aligned
+constexpr uint32_t B_BYTES = BN * BK_BYTES;                 // 32 KB
+constexpr uint32_t SF_TILE = 512;                           // one 128-row x 4-block scale tile
+constexpr uint32_t SFA_BYTES = KB_PER_STAGE * SF_TILE;      // 2 KB
+constexpr uint32_t SFB_BYTES = 2 * KB_PER_STAGE * SF_TILE;  // 4 KB (two 128-row tiles)
+constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;  // 54 KB
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t SF_COL0 = 2 * BN;                        // scale factors after both accumulators
-constexpr uint32_t SF_BUF_COLS = 4 * KB_PER_STAGE + 8 * KB_PER_STAGE;  // 16 (A) + 32 (B)
-constexpr int NUM_THREADS = 192;
-constexpr uint32_t SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+constexpr uint32_t SF_COL0 = BN;                            // scale buffers after the accumulator
+constexpr uint32_t SF_BUF_COLS = 4 * KB_PER_STAGE + 8 * KB_PER_STAGE;  // 16 (A) + 32 (B) per stage
+constexpr int NUM_THREADS = 384;
+constexpr int EPI_WARP0 = 4;
+constexpr int EPI_THREADS = 256;
+constexpr uint32_t SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 5120 /*barriers, alpha*/;
 constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;           // 2 s per wait
 
-static_assert(SF_COL0 + 2 * SF_BUF_COLS <= TMEM_COLS, "TMEM budget");
+static_assert(SF_COL0 + STAGES * SF_BUF_COLS <= TMEM_COLS, "TMEM budget");
 static_assert(STAGE_BYTES % 1024 == 0, "stage alignment for the 128-byte swizzle");
 
 // Instruction descriptor: dense, A/B = E2M1 (kind::mxf4nvf4 format 1),
-// K-major A and B, scale format UE4M3, N = 192 (>>3), M = 128 (>>4).
-constexpr uint32_t IDESC = (1u << 7) | (1u << 10) | (uint32_t(BN >> 3) << 17) | (uint32_t(BM >> 4) << 24);
+// K-major A and B, scale format UE4M3, N = 128 (>>3), M = 128 (>>4).
+constexpr uint32_t IDESC = (1u << 7) | (1u << 10) | (uint32_t(HALF_N >> 3) << 17) | (uint32_t(BM >> 4) << 24);
 
 struct Params {
     int32_t M, N, K;
@@ -80,11 +89,13 @@ struct Params {
 struct Smem {
     uint64_t full[STAGES];
     uint64_t empty[STAGES];
-    uint64_t acc_full[2];
-    uint64_t acc_empty[2];
+    uint64_t sf_ready[STAGES];
+    uint64_t acc_full;
+    uint64_t acc_empty;
     uint64_t drain;
     uint32_t tmem_base;
     volatile int32_t abort_flag;
+    float alpha[EPI_THREADS / 32][HALF_N];  // per epilogue warp: alpha of its 128 columns
 };
 
 __device__ __forceinline__ void raise_timeout(Smem *sm, uint32_t *status)
@@ -104,41 +115,53 @@ __device__ __forceinline__ float column_alpha(const Params &p, float ga, int32_t
     return __fmul_rn(ga, __ldg(p.g_w + s));
 }
 
-__device__ __forceinline__ void store_chunk(const Params &p, int32_t row, int32_t col0, const float (&f)[32])
+// Scale 64 accumulator columns by alpha and store them for one row.
+__device__ __forceinline__ void store_64(const Params &p, const float *alpha, int32_t row, int32_t col0,
+                                         const uint32_t (&v)[64])
 {
-    if (row >= p.M)
+    if (row >= p.M || col0 >= p.N)
         return;
     const int64_t off = static_cast<int64_t>(row) * p.N + col0;
-    const bool full = p.vec_ok && (col0 + 32 <= p.N);
+    const bool full = p.vec_ok && (col0 + 64 <= p.N);
     if (p.out_fp32) {
         float *o = static_cast<float *>(p.out) + off;
         if (full) {
 #pragma unroll
-            for (int j = 0; j < 32; j += 4)
-                *reinterpret_cast<float4 *>(o + j) = make_float4(f[j], f[j + 1], f[j + 2], f[j + 3]);
+            for (int j = 0; j < 64; j += 4) {
+                const float4 a = *reinterpret_cast<const float4 *>(&alpha[j]);
+                *reinterpret_cast<float4 *>(o + j) =
+                    make_float4(__fmul_rn(__uint_as_float(v[j]), a.x), __fmul_rn(__uint_as_float(v[j + 1]), a.y),
+                                __fmul_rn(__uint_as_float(v[j + 2]), a.z), __fmul_rn(__uint_as_float(v[j + 3]), a.w));
+            }
         } else {
-            for (int j = 0; j < 32 && col0 + j < p.N; ++j)
-                o[j] = f[j];
+            for (int j = 0; j < 64 && col0 + j < p.N; ++j)
+                o[j] = __fmul_rn(__uint_as_float(v[j]), alpha[j]);
         }
     } else {
         __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(p.out) + off;
         if (full) {
 #pragma unroll
-            for (int j = 0; j < 32; j += 8) {
-                uint4 v;
-                __nv_bfloat162 b0 = __floats2bfloat162_rn(f[j], f[j + 1]);
-                __nv_bfloat162 b1 = __floats2bfloat162_rn(f[j + 2], f[j + 3]);
-                __nv_bfloat162 b2 = __floats2bfloat162_rn(f[j + 4], f[j + 5]);
-                __nv_bfloat162 b3 = __floats2bfloat162_rn(f[j + 6], f[j + 7]);
-                v.x = *reinterpret_cast<uint32_t *>(&b0);
-                v.y = *reinterpret_cast<uint32_t *>(&b1);
-                v.z = *reinterpret_cast<uint32_t *>(&b2);
-                v.w = *reinterpret_cast<uint32_t *>(&b3);
-                *reinterpret_cast<uint4 *>(o + j) = v;
+            for (int j = 0; j < 64; j += 8) {
+                const float4 a0 = *reinterpret_cast<const float4 *>(&alpha[j]);
+                const float4 a1 = *reinterpret_cast<const float4 *>(&alpha[j + 4]);
+                __nv_bfloat162 b0 = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(v[j]), a0.x),
+                                                          __fmul_rn(__uint_as_float(v[j + 1]), a0.y));
+                __nv_bfloat162 b1 = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(v[j + 2]), a0.z),
+                                                          __fmul_rn(__uint_as_float(v[j + 3]), a0.w));
+                __nv_bfloat162 b2 = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(v[j + 4]), a1.x),
+                                                          __fmul_rn(__uint_as_float(v[j + 5]), a1.y));
+                __nv_bfloat162 b3 = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(v[j + 6]), a1.z),
+                                                          __fmul_rn(__uint_as_float(v[j + 7]), a1.w));
+                uint4 w;
+                w.x = *reinterpret_cast<uint32_t *>(&b0);
+                w.y = *reinterpret_cast<uint32_t *>(&b1);
+                w.z = *reinterpret_cast<uint32_t *>(&b2);
+                w.w = *reinterpret_cast<uint32_t *>(&b3);
+                *reinterpret_cast<uint4 *>(o + j) = w;
             }
         } else {
-            for (int j = 0; j < 32 && col0 + j < p.N; ++j)
-                o[j] = __float2bfloat16_rn(f[j]);
+            for (int j = 0; j < 64 && col0 + j < p.N; ++j)
+                o[j] = __float2bfloat16_rn(__fmul_rn(__uint_as_float(v[j]), alpha[j]));
         }
     }
 }
@@ -163,11 +186,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(smem_u32(&sm->full[s]), 1);
             mbar_init(smem_u32(&sm->empty[s]), 1);
+            mbar_init(smem_u32(&sm->sf_ready[s]), 1);
         }
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(smem_u32(&sm->acc_full[b]), 1);
-            mbar_init(smem_u32(&sm->acc_empty[b]), 4);
-        }
+        mbar_init(smem_u32(&sm->acc_full), 1);
+        mbar_init(smem_u32(&sm->acc_empty), EPI_THREADS / 32);
         mbar_init(smem_u32(&sm->drain), 1);
         sm->abort_flag = 0;
         fence_mbarrier_init();
@@ -193,7 +215,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             for (int tile = blockIdx.x; tile < p.num_tiles && !sm->abort_flag; tile += gridDim.x) {
                 const int m_blk = tile % p.num_m, n_blk = tile / p.num_m;
                 const int m0 = m_blk * BM, n0 = n_blk * BN;
-                const int rb0 = n0 >> 7;
+                const int rb0 = n0 >> 7;  // first 128-row scale tile of W
                 const int nb_tiles = (rb0 + 1 < p.n_row_tiles) ? 2 : 1;
                 for (int kt = 0; kt < p.kt_total; ++kt) {
                     if (!mbar_wait_bounded(smem_u32(&sm->empty[stage]), phase ^ 1u, WAIT_LIMIT_NS)) {
@@ -201,17 +223,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                         break;
                     }
                     const int nkb = min(KB_PER_STAGE, p.kb_total - kt * KB_PER_STAGE);
-                    const uint32_t sf_bytes = nkb * 512u;
+                    const uint32_t sf_bytes = nkb * SF_TILE;
                     const uint32_t bar = smem_u32(&sm->full[stage]);
                     mbar_arrive_expect_tx(bar, A_BYTES + B_BYTES + sf_bytes * (1 + nb_tiles));
                     tma_load_2d(a_smem(stage), &tmA, kt * BK_BYTES, m0, bar);
                     tma_load_2d(b_smem(stage), &tmB, kt * BK_BYTES, n0, bar);
                     bulk_load(sfa_smem(stage),
-                              p.sfa + (static_cast<int64_t>(m_blk) * p.kb_total + kt * KB_PER_STAGE) * 512,
+                              p.sfa + (static_cast<int64_t>(m_blk) * p.kb_total + kt * KB_PER_STAGE) * SF_TILE,
                               sf_bytes, bar);
                     for (int j = 0; j < nb_tiles; ++j)
-                        bulk_load(sfb_smem(stage) + j * (KB_PER_STAGE * 512),
-                                  p.sfb + (static_cast<int64_t>(rb0 + j) * p.kb_total + kt * KB_PER_STAGE) * 512,
+                        bulk_load(sfb_smem(stage) + j * (KB_PER_STAGE * SF_TILE),
+                                  p.sfb + (static_cast<int64_t>(rb0 + j) * p.kb_total + kt * KB_PER_STAGE) * SF_TILE,
                                   sf_bytes, bar);
                     if (++stage == STAGES) {
                         stage = 0;
@@ -225,42 +247,35 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (lane == 0) {
             int stage = 0;
             uint32_t phase = 0;
-            uint32_t sf_buf = 0;
             int local = 0;
             for (int tile = blockIdx.x; tile < p.num_tiles && !sm->abort_flag; tile += gridDim.x, ++local) {
-                const int n0 = (tile / p.num_m) * BN;
-                const uint32_t sfb_shift = (n0 & 127) >> 5;  // 0 or 2 columns: first W row of the tile
-                const int acc = local & 1;
-                const uint32_t acc_phase = (local >> 1) & 1;
-                if (!mbar_wait_bounded(smem_u32(&sm->acc_empty[acc]), acc_phase ^ 1u, WAIT_LIMIT_NS)) {
+                if (!mbar_wait_bounded(smem_u32(&sm->acc_empty), (local & 1) ^ 1u, WAIT_LIMIT_NS)) {
                     raise_timeout(sm, p.status);
                     break;
                 }
                 tc_fence_after();
-                const uint32_t d_tmem = tmem + acc * BN;
                 bool ok = true;
                 for (int kt = 0; kt < p.kt_total; ++kt) {
-                    if (!mbar_wait_bounded(smem_u32(&sm->full[stage]), phase, WAIT_LIMIT_NS)) {
+                    if (!mbar_wait_bounded(smem_u32(&sm->full[stage]), phase, WAIT_LIMIT_NS) ||
+                        !mbar_wait_bounded(smem_u32(&sm->sf_ready[stage]), phase, WAIT_LIMIT_NS)) {
                         raise_timeout(sm, p.status);
                         ok = false;
                         break;
                     }
                     tc_fence_after();
                     const int nkb = min(KB_PER_STAGE, p.kb_total - kt * KB_PER_STAGE);
-                    const uint32_t sfa_t = tmem + SF_COL0 + sf_buf * SF_BUF_COLS;
+                    const uint32_t sfa_t = tmem + SF_COL0 + stage * SF_BUF_COLS;
                     const uint32_t sfb_t = sfa_t + 4 * KB_PER_STAGE;
-                    sf_buf ^= 1u;
-                    for (int kb = 0; kb < nkb; ++kb) {
-                        tc_cp_32x128b_x4(sfa_t + kb * 4, smem_desc(sfa_smem(stage) + kb * 512, 0, 128, 0));
-                        tc_cp_32x128b_x4(sfb_t + kb * 8, smem_desc(sfb_smem(stage) + kb * 512, 0, 128, 0));
-                        tc_cp_32x128b_x4(sfb_t + kb * 8 + 4,
-                                         smem_desc(sfb_smem(stage) + KB_PER_STAGE * 512 + kb * 512, 0, 128, 0));
-                    }
                     for (int kb = 0; kb < nkb; ++kb) {
                         const uint64_t adesc = smem_desc(a_smem(stage) + kb * 32, 16, 1024, 2);
-                        const uint64_t bdesc = smem_desc(b_smem(stage) + kb * 32, 16, 1024, 2);
-                        tc_mma_nvf4(d_tmem, adesc, bdesc, IDESC, sfa_t + kb * 4, sfb_t + kb * 8 + sfb_shift,
-                                    (kt > 0 || kb > 0) ? 1u : 0u);
+                        const uint32_t acc_flag = (kt > 0 || kb > 0) ? 1u : 0u;
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            const uint64_t bdesc =
+                                smem_desc(b_smem(stage) + h * (HALF_N * BK_BYTES) + kb * 32, 16, 1024, 2);
+                            tc_mma_nvf4(tmem + h * HALF_N, adesc, bdesc, IDESC, sfa_t + kb * 4,
+                                        sfb_t + kb * 8 + h * 4, acc_flag);
+                        }
                     }
                     tc_commit(smem_u32(&sm->empty[stage]));
                     if (++stage == STAGES) {
@@ -270,47 +285,82 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 }
                 if (!ok)
                     break;
-                tc_commit(smem_u32(&sm->acc_full[acc]));
+                tc_commit(smem_u32(&sm->acc_full));
             }
             // let every tcgen05 operation this thread issued finish before TMEM is freed
             tc_commit(smem_u32(&sm->drain));
             if (!mbar_wait_bounded(smem_u32(&sm->drain), 0, WAIT_LIMIT_NS))
                 raise_timeout(sm, p.status);
         }
-    } else {
+    } else if (warp == 2) {
+        // ------------------------------------- scale factors -> TMEM
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            for (int tile = blockIdx.x; tile < p.num_tiles && !sm->abort_flag; tile += gridDim.x) {
+                bool ok = true;
+                for (int kt = 0; kt < p.kt_total; ++kt) {
+                    // The stage's TMEM scale buffer is free: the producer only refilled this
+                    // stage after the MMAs that read the buffer last time had completed.
+                    if (!mbar_wait_bounded(smem_u32(&sm->full[stage]), phase, WAIT_LIMIT_NS)) {
+                        raise_timeout(sm, p.status);
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const int nkb = min(KB_PER_STAGE, p.kb_total - kt * KB_PER_STAGE);
+                    const uint32_t sfa_t = tmem + SF_COL0 + stage * SF_BUF_COLS;
+                    const uint32_t sfb_t = sfa_t + 4 * KB_PER_STAGE;
+                    for (int kb = 0; kb < nkb; ++kb) {
+                        tc_cp_32x128b_x4(sfa_t + kb * 4, smem_desc(sfa_smem(stage) + kb * SF_TILE, 0, 128, 0));
+                        tc_cp_32x128b_x4(sfb_t + kb * 8, smem_desc(sfb_smem(stage) + kb * SF_TILE, 0, 128, 0));
+                        tc_cp_32x128b_x4(sfb_t + kb * 8 + 4,
+                                         smem_desc(sfb_smem(stage) + (KB_PER_STAGE + kb) * SF_TILE, 0, 128, 0));
+                    }
+                    tc_commit(smem_u32(&sm->sf_ready[stage]));
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok)
+                    break;
+            }
+        }
+    } else if (warp >= EPI_WARP0) {
         // ------------------------------------------------------ epilogue
-        const int q = warp & 3;  // TMEM lane quarter this warp may access
+        const int q = warp & 3;                    // TMEM lane quarter this warp may access
+        const int hc = (warp - EPI_WARP0) >> 2;    // which 128-column half of the tile
+        float *alpha = sm->alpha[warp - EPI_WARP0];
         const float ga = __ldg(p.g_a);
         int local = 0;
         for (int tile = blockIdx.x; tile < p.num_tiles && !sm->abort_flag; tile += gridDim.x, ++local) {
             const int m0 = (tile % p.num_m) * BM, n0 = (tile / p.num_m) * BN;
-            const int acc = local & 1;
-            const uint32_t acc_phase = (local >> 1) & 1;
-            if (!mbar_wait_bounded(smem_u32(&sm->acc_full[acc]), acc_phase, WAIT_LIMIT_NS)) {
-                raise_timeout(sm, p.status);
+            __syncwarp();  // this warp's reads of the previous tile's alpha are done
+#pragma unroll
+            for (int j = 0; j < HALF_N / 32; ++j)
+                alpha[lane + 32 * j] = column_alpha(p, ga, n0 + hc * HALF_N + lane + 32 * j);
+            __syncwarp();
+            // every lane waits (bounded); the vote keeps the warp's decision uniform
+            const bool ok = mbar_wait_bounded(smem_u32(&sm->acc_full), local & 1, WAIT_LIMIT_NS);
+            if (!__all_sync(0xFFFFFFFFu, ok)) {
+                if (lane == 0)
+                    raise_timeout(sm, p.status);
                 break;
             }
             tc_fence_after();
+            const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16) + hc * HALF_N;
+            uint32_t v0[64], v1[64];
+            tc_ld_32x32b_x64(taddr, v0);
+            tc_ld_32x32b_x64(taddr + 64, v1);
+            tc_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(smem_u32(&sm->acc_empty));
             const int row = m0 + q * 32 + lane;
-#pragma unroll 1
-            for (int c = 0; c < BN / 32; ++c) {
-                uint32_t v[32];
-                tc_ld_32x32b_x32(tmem + (static_cast<uint32_t>(q * 32) << 16) + acc * BN + c * 32, v);
-                tc_wait_ld();
-                if (c == BN / 32 - 1) {
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0)
-                        mbar_arrive(smem_u32(&sm->acc_empty[acc]));
-                }
-                const int col0 = n0 + c * 32;
-                const float al = column_alpha(p, ga, col0 + lane);
-                float f[32];
-#pragma unroll
-                for (int j = 0; j < 32; ++j)
-                    f[j] = __fmul_rn(__uint_as_float(v[j]), __shfl_sync(0xFFFFFFFFu, al, j));
-                store_chunk(p, row, col0, f);
-            }
+            store_64(p, alpha, row, n0 + hc * HALF_N, v0);
+            store_64(p, alpha + 64, row, n0 + hc * HALF_N + 64, v1);
         }
     }
 

@@ -212,7 +212,7 @@ int check_gemm_shape(int64_t M, int64_t N, int64_t K)
     if (K % 64 != 0)
         return NVFP4_ERR_UNSUPPORTED_SHAPE;
     if (M > (int64_t(1) << 30) || N > (int64_t(1) << 30) || K > (int64_t(1) << 30) ||
-        cdiv(M, 128) * cdiv(N, 192) >= (int64_t(1) << 31))
+        cdiv(M, nvfp4::gemm::BM) * cdiv(N, nvfp4::gemm::BN) >= (int64_t(1) << 31))
         return NVFP4_ERR_UNSUPPORTED_SHAPE;
     return NVFP4_OK;
 }
