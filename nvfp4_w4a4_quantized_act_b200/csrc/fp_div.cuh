@@ -1,0 +1,43 @@
+// fp_div.cuh -- correctly rounded division of many dividends by one shared
+// divisor, for the block quantizer (the 16 elements of a block all divide by
+// the block's decode scale d = fl32(s * g)).
+//
+// Method: with r = RN(1/d) computed once (CUDA's correctly rounded
+// reciprocal), each quotient is
+//     q = RN(x * r),  e = x - d*q  (exact, one fused multiply-add),
+//     y = RN(q + e*r)              (one fused multiply-add),
+// the final correction step of P. Markstein, "Computation of elementary
+// functions on the IBM RISC System/6000 processor", IBM J. Res. Develop.
+// 34(1), 1990: when r is the correctly rounded reciprocal and q is within one
+// ulp of x/d, y is the correctly rounded quotient, provided nothing leaves the
+// normal range.  div_shared_ok() checks the divisor once per block; outside
+// that range the caller uses the plain IEEE division.  With d >= 2^-80 the
+// remainder e is exact whenever |x| >= 2^-103, so every quotient of magnitude
+// >= 2^-20 is the IEEE one; smaller quotients (from dividends near the bottom
+// of the fp32 range) may differ in their last bits but stay far below 0.25,
+// where every one of them encodes to the same E2M1 code, +-0 by the sign of x.
+// The sign is copied from x so that -0 / d stays -0 as in IEEE division.
+// tests/test_division_gpu.py compares this routine with __fdiv_rn over every
+// pair of bf16 and fp32 significands and over the whole accepted range.
+#pragma once
+
+#include <cstdint>
+
+namespace nvfp4 {
+
+// d is normal and far from both ends of the exponent range, and every
+// |x| <= bound keeps x / d below 2^100.
+__device__ __forceinline__ bool div_shared_ok(float d, float bound)
+{
+    return d >= 0x1p-80f && d <= 0x1p100f && bound <= __fmul_rn(d, 0x1p100f);
+}
+
+__device__ __forceinline__ float div_shared(float x, float d, float r)
+{
+    const float q = __fmul_rn(x, r);
+    const float e = __fmaf_rn(-d, q, x);
+    const float y = __fmaf_rn(e, r, q);
+    return __uint_as_float((__float_as_uint(y) & 0x7FFFFFFFu) | (__float_as_uint(x) & 0x80000000u));
+}
+
+}  // namespace nvfp4

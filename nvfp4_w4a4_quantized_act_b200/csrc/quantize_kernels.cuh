@@ -23,6 +23,7 @@
 #include <cstdint>
 #include <cuda_bf16.h>
 
+#include "fp_div.cuh"
 #include "ptx_sm100.cuh"
 
 namespace nvfp4 {
@@ -143,15 +144,26 @@ __device__ __forceinline__ float global_scale_from_amax(uint32_t bits)
 // One thread per 16-element block; four consecutive threads cover the four
 // blocks that share one 32-bit scale word.  Grid-stride over
 // rows_pad * groups * 4 threads (rows past `rows` only write zero scales).
+// Elements divide by the block's decode scale d with div_shared() (exact
+// IEEE quotient from one reciprocal per block), falling back to the IEEE
+// division for blocks whose d is near the ends of the exponent range.
 __global__ void __launch_bounds__(256) quantize_kernel(const QuantParams p)
 {
+    __shared__ float s_g[kMaxSeg];
+    if (threadIdx.x < p.seg.nseg) {
+        const float g = (p.mode == 0) ? global_scale_from_amax(p.amax_bits[threadIdx.x]) : p.g_in[threadIdx.x];
+        s_g[threadIdx.x] = g;
+        if (p.mode == 0 && p.g_out != nullptr && blockIdx.x == 0)
+            p.g_out[threadIdx.x] = g;
+    }
+    __syncthreads();
+
     const uint32_t total = static_cast<uint32_t>(p.rows_pad) * static_cast<uint32_t>(p.groups) * 4u;
     const uint32_t stride = gridDim.x * blockDim.x;
     const int lane = threadIdx.x & 31;
     const int nblk = p.K >> 4;
-
-    if (p.mode == 0 && p.g_out != nullptr && blockIdx.x == 0 && threadIdx.x < p.seg.nseg)
-        p.g_out[threadIdx.x] = global_scale_from_amax(p.amax_bits[threadIdx.x]);
+    const bool one_seg = p.seg.nseg == 1;
+    const float g_first = s_g[0];
 
     // Loop bound is warp-uniform so every lane takes part in the shuffles.
     for (uint32_t base = blockIdx.x * blockDim.x + (threadIdx.x & ~31u); base < total; base += stride) {
@@ -162,12 +174,7 @@ __global__ void __launch_bounds__(256) quantize_kernel(const QuantParams p)
         const int blk = static_cast<int>(cg * 4u + sub);
         uint32_t sbyte = 0;
         if (t < total && row < static_cast<uint32_t>(p.rows) && blk < nblk) {
-            float g;
-            const int s = seg_of(p.seg, row);
-            if (p.mode == 0)
-                g = global_scale_from_amax(p.amax_bits[s]);
-            else
-                g = p.g_in[s];
+            const float g = one_seg ? g_first : s_g[seg_of(p.seg, row)];
             const uint4 *src = reinterpret_cast<const uint4 *>(p.X + static_cast<int64_t>(row) * p.ld + blk * 16);
             const uint4 v0 = __ldg(src), v1 = __ldg(src + 1);
             const uint32_t bmax = hmax16(vmax_mag(vmax_mag(0u, v0), v1));
@@ -183,6 +190,14 @@ __global__ void __launch_bounds__(256) quantize_kernel(const QuantParams p)
                 for (int i = 0; i < 8; ++i) {
                     const uint32_t lo = (w[i] >> 15) & 1u, hi = (w[i] >> 31) & 1u;
                     packed[i >> 2] |= ((lo << 3) | (hi << 7)) << ((i & 3) * 8);
+                }
+            } else if (div_shared_ok(d, bamax)) {
+                const float r = __frcp_rn(d);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const float y0 = div_shared(bf16_lo(w[i]), d, r);
+                    const float y1 = div_shared(bf16_hi(w[i]), d, r);
+                    packed[i >> 2] |= f32x2_to_e2m1x2(y0, y1) << ((i & 3) * 8);
                 }
             } else {
 #pragma unroll
