@@ -16,7 +16,6 @@
 // >= 2^-20 is the IEEE one; smaller quotients (from dividends near the bottom
 // of the fp32 range) may differ in their last bits but stay far below 0.25,
 // where every one of them encodes to the same E2M1 code, +-0 by the sign of x.
-// The sign is copied from x so that -0 / d stays -0 as in IEEE division.
 // tests/test_division_gpu.py compares this routine with __fdiv_rn over every
 // pair of bf16 and fp32 significands and over the whole accepted range.
 #pragma once
@@ -34,10 +33,12 @@ __device__ __forceinline__ bool div_shared_ok(float d, float bound)
 
 __device__ __forceinline__ float div_shared(float x, float d, float r)
 {
+    // e' = d*q - x = -e.  Written this way round, x = -0 gives q = -0,
+    // e' = (-0) + (+0) = +0 and y = (-0) + (-0) = -0: the IEEE sign of zero
+    // comes out of the arithmetic without a separate sign fix-up.
     const float q = __fmul_rn(x, r);
-    const float e = __fmaf_rn(-d, q, x);
-    const float y = __fmaf_rn(e, r, q);
-    return __uint_as_float((__float_as_uint(y) & 0x7FFFFFFFu) | (__float_as_uint(x) & 0x80000000u));
+    const float en = __fmaf_rn(d, q, -x);
+    return __fmaf_rn(-en, r, q);
 }
 
 }  // namespace nvfp4

@@ -47,10 +47,13 @@ __device__ __forceinline__ int seg_of(const SegRows &s, int64_t r)
     return k;
 }
 
-// Packed max of the magnitudes (sign cleared) of the two bf16 in `w`.
+// Packed max of the magnitudes of the two bf16 in `w`, each kept as
+// (magnitude << 1) in its 16-bit half: w + w pushes the upper sign bit out
+// and the lower sign bit into the upper half's lowest bit, which hmax16()
+// shifts away again.
 __device__ __forceinline__ uint32_t vmax_mag(uint32_t acc, uint32_t w)
 {
-    return __vmaxu2(acc, w & 0x7FFF7FFFu);
+    return __vmaxu2(acc, w + w);
 }
 
 __device__ __forceinline__ uint32_t vmax_mag(uint32_t acc, const uint4 &v)
@@ -62,7 +65,8 @@ __device__ __forceinline__ uint32_t vmax_mag(uint32_t acc, const uint4 &v)
     return acc;
 }
 
-__device__ __forceinline__ uint32_t hmax16(uint32_t packed) { return max(packed & 0xFFFFu, packed >> 16); }
+// Largest bf16 magnitude (bits, sign cleared) of a vmax_mag() accumulator.
+__device__ __forceinline__ uint32_t hmax16(uint32_t packed) { return max(packed & 0xFFFFu, packed >> 16) >> 1; }
 
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
@@ -141,87 +145,123 @@ __device__ __forceinline__ float global_scale_from_amax(uint32_t bits)
     return a == 0.0f ? 1.0f : __fdiv_rn(a, 2688.0f);
 }
 
-// One thread per 16-element block; four consecutive threads cover the four
-// blocks that share one 32-bit scale word.  Grid-stride over
-// rows_pad * groups * 4 threads (rows past `rows` only write zero scales).
-// Elements divide by the block's decode scale d with div_shared() (exact
-// IEEE quotient from one reciprocal per block), falling back to the IEEE
-// division for blocks whose d is near the ends of the exponent range.
+// Block scale and codes of one 16-element block held as two 16-byte words.
+// Returns the E4M3 scale byte and writes the 8 code bytes to packed[0..1].
+__device__ __forceinline__ uint32_t quantize_block(const uint4 &v0, const uint4 &v1, float g, float rg, bool g_ok,
+                                                   uint32_t (&packed)[2])
+{
+    const uint32_t bmax = hmax16(vmax_mag(vmax_mag(0u, v0), v1));
+    const float bamax = __uint_as_float(bmax << 16);
+    // s32 = fl32(fl32(bamax / 6) / g), by the shared-divisor division where it is exact
+    float s32;
+    const float t_fast = div_shared(bamax, 6.0f, 0x1.555556p-3f /* RN(1/6) */);
+    if (g_ok && bamax >= 0x1p-17f && bamax <= 0x1p100f && div_shared_ok(g, t_fast))
+        s32 = div_shared(t_fast, g, rg);
+    else
+        s32 = __fdiv_rn(__fdiv_rn(bamax, 6.0f), g);
+    const uint32_t sbyte = f32_to_e4m3_satfinite(s32);
+    const float d = __fmul_rn(e4m3_to_f32(sbyte), g);
+    const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+    packed[0] = packed[1] = 0u;
+    if (d == 0.0f) {
+        // zero scale: every code is +-0 with the sign of its input
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const uint32_t lo = (w[i] >> 15) & 1u, hi = (w[i] >> 31) & 1u;
+            packed[i >> 2] |= ((lo << 3) | (hi << 7)) << ((i & 3) * 8);
+        }
+    } else if (div_shared_ok(d, bamax)) {
+        const float r = __frcp_rn(d);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const float y0 = div_shared(bf16_lo(w[i]), d, r);
+            const float y1 = div_shared(bf16_hi(w[i]), d, r);
+            packed[i >> 2] |= f32x2_to_e2m1x2(y0, y1) << ((i & 3) * 8);
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const float y0 = __fdiv_rn(bf16_lo(w[i]), d);
+            const float y1 = __fdiv_rn(bf16_hi(w[i]), d);
+            packed[i >> 2] |= f32x2_to_e2m1x2(y0, y1) << ((i & 3) * 8);
+        }
+    }
+    return sbyte;
+}
+
+// Work item = one 512-element chunk of one row (32 blocks = 8 scale words),
+// one lane per 16-element block.  Warps stride over the rows_pad x chunks
+// items; the next item's input is loaded before the current one is
+// quantized.  Rows past `rows` (up to the 128-row padding) and blocks past K
+// only write zero scale bytes.
 __global__ void __launch_bounds__(256) quantize_kernel(const QuantParams p)
 {
-    __shared__ float s_g[kMaxSeg];
+    __shared__ float s_g[kMaxSeg], s_rg[kMaxSeg];
+    __shared__ int s_gok[kMaxSeg];
     if (threadIdx.x < p.seg.nseg) {
         const float g = (p.mode == 0) ? global_scale_from_amax(p.amax_bits[threadIdx.x]) : p.g_in[threadIdx.x];
         s_g[threadIdx.x] = g;
+        s_rg[threadIdx.x] = __frcp_rn(g);
+        s_gok[threadIdx.x] = (g >= 0x1p-80f && g <= 0x1p100f) ? 1 : 0;
         if (p.mode == 0 && p.g_out != nullptr && blockIdx.x == 0)
             p.g_out[threadIdx.x] = g;
     }
     __syncthreads();
 
-    const uint32_t total = static_cast<uint32_t>(p.rows_pad) * static_cast<uint32_t>(p.groups) * 4u;
-    const uint32_t stride = gridDim.x * blockDim.x;
     const int lane = threadIdx.x & 31;
+    const uint32_t cpr = (static_cast<uint32_t>(p.groups) + 7u) >> 3;  // chunks per row
+    const uint32_t items = static_cast<uint32_t>(p.rows_pad) * cpr;
+    const uint32_t warp0 = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const uint32_t nwarps = (gridDim.x * blockDim.x) >> 5;
+    const uint32_t drow = nwarps / cpr, dchunk = nwarps - drow * cpr;
     const int nblk = p.K >> 4;
     const bool one_seg = p.seg.nseg == 1;
-    const float g_first = s_g[0];
 
-    // Loop bound is warp-uniform so every lane takes part in the shuffles.
-    for (uint32_t base = blockIdx.x * blockDim.x + (threadIdx.x & ~31u); base < total; base += stride) {
-        const uint32_t t = base + lane;
-        const uint32_t u = t >> 2, sub = t & 3u;
-        const uint32_t row = u / static_cast<uint32_t>(p.groups);
-        const uint32_t cg = u - row * static_cast<uint32_t>(p.groups);
-        const int blk = static_cast<int>(cg * 4u + sub);
-        uint32_t sbyte = 0;
-        if (t < total && row < static_cast<uint32_t>(p.rows) && blk < nblk) {
-            const float g = one_seg ? g_first : s_g[seg_of(p.seg, row)];
-            const uint4 *src = reinterpret_cast<const uint4 *>(p.X + static_cast<int64_t>(row) * p.ld + blk * 16);
-            const uint4 v0 = __ldg(src), v1 = __ldg(src + 1);
-            const uint32_t bmax = hmax16(vmax_mag(vmax_mag(0u, v0), v1));
-            const float bamax = __uint_as_float(bmax << 16);
-            const float s32 = __fdiv_rn(__fdiv_rn(bamax, 6.0f), g);
-            sbyte = f32_to_e4m3_satfinite(s32);
-            const float d = __fmul_rn(e4m3_to_f32(sbyte), g);
-            const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-            uint32_t packed[2] = {0u, 0u};
-            if (d == 0.0f) {
-                // zero scale: every code is +-0 with the sign of its input
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const uint32_t lo = (w[i] >> 15) & 1u, hi = (w[i] >> 31) & 1u;
-                    packed[i >> 2] |= ((lo << 3) | (hi << 7)) << ((i & 3) * 8);
-                }
-            } else if (div_shared_ok(d, bamax)) {
-                const float r = __frcp_rn(d);
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const float y0 = div_shared(bf16_lo(w[i]), d, r);
-                    const float y1 = div_shared(bf16_hi(w[i]), d, r);
-                    packed[i >> 2] |= f32x2_to_e2m1x2(y0, y1) << ((i & 3) * 8);
-                }
-            } else {
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const float y0 = __fdiv_rn(bf16_lo(w[i]), d);
-                    const float y1 = __fdiv_rn(bf16_hi(w[i]), d);
-                    packed[i >> 2] |= f32x2_to_e2m1x2(y0, y1) << ((i & 3) * 8);
-                }
-            }
-            uint2 *dst = reinterpret_cast<uint2 *>(p.codes + static_cast<int64_t>(row) * (p.K >> 1) + blk * 8);
-            *dst = make_uint2(packed[0], packed[1]);
+    uint32_t row = warp0 / cpr, chunk = warp0 - row * cpr;
+    auto load = [&](uint32_t r, uint32_t c, uint4 &a, uint4 &b) {
+        const int blk = static_cast<int>(c * 32u) + lane;
+        if (r < static_cast<uint32_t>(p.rows) && blk < nblk) {
+            const uint4 *src = reinterpret_cast<const uint4 *>(p.X + static_cast<int64_t>(r) * p.ld + blk * 16);
+            a = __ldg(src);
+            b = __ldg(src + 1);
         }
-        // gather the four scale bytes of this group into lane (lane & ~3)
-        const int g0 = lane & ~3;
-        const uint32_t b0 = __shfl_sync(0xFFFFFFFFu, sbyte, g0);
-        const uint32_t b1 = __shfl_sync(0xFFFFFFFFu, sbyte, g0 + 1);
-        const uint32_t b2 = __shfl_sync(0xFFFFFFFFu, sbyte, g0 + 2);
-        const uint32_t b3 = __shfl_sync(0xFFFFFFFFu, sbyte, g0 + 3);
-        if (sub == 0 && t < total) {
-            const uint32_t word = b0 | (b1 << 8) | (b2 << 16) | (b3 << 24);
+    };
+    uint4 v0 = make_uint4(0, 0, 0, 0), v1 = v0;
+    if (warp0 < items)
+        load(row, chunk, v0, v1);
+    for (uint32_t item = warp0; item < items; item += nwarps) {
+        // advance to the next item and start its loads
+        uint32_t nrow = row + drow, nchunk = chunk + dchunk;
+        if (nchunk >= cpr) {
+            nchunk -= cpr;
+            ++nrow;
+        }
+        uint4 n0 = make_uint4(0, 0, 0, 0), n1 = n0;
+        if (item + nwarps < items)
+            load(nrow, nchunk, n0, n1);
+
+        const int blk = static_cast<int>(chunk * 32u) + lane;
+        uint32_t sbyte = 0;
+        if (row < static_cast<uint32_t>(p.rows) && blk < nblk) {
+            const int sg = one_seg ? 0 : seg_of(p.seg, row);
+            uint32_t packed[2];
+            sbyte = quantize_block(v0, v1, s_g[sg], s_rg[sg], s_gok[sg] != 0, packed);
+            *reinterpret_cast<uint2 *>(p.codes + static_cast<int64_t>(row) * (p.K >> 1) + blk * 8) =
+                make_uint2(packed[0], packed[1]);
+        }
+        // four neighbouring blocks -> one 32-bit scale word, in lanes 0, 4, 8, ...
+        const uint32_t pair = sbyte | (__shfl_down_sync(0xFFFFFFFFu, sbyte, 1) << 8);
+        const uint32_t word = pair | (__shfl_down_sync(0xFFFFFFFFu, pair, 2) << 16);
+        const uint32_t cg = chunk * 8u + (lane >> 2);
+        if ((lane & 3) == 0 && cg < static_cast<uint32_t>(p.groups)) {
             const uint64_t tile = static_cast<uint64_t>(row >> 7) * p.groups + cg;
             const uint32_t rr = row & 127u;
             *reinterpret_cast<uint32_t *>(p.sf + tile * 512 + (rr & 31u) * 16 + (rr >> 5) * 4) = word;
         }
+        row = nrow;
+        chunk = nchunk;
+        v0 = n0;
+        v1 = n1;
     }
 }
 
