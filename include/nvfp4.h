@@ -166,6 +166,40 @@ int nvfp4_swiglu_quantize(const void *gate_up, int64_t M, int64_t F, int64_t ld,
                           void *h, uint8_t *codes, uint8_t *sf, float *g_h,
                           void *ws, size_t ws_bytes, void *stream);
 
+/* Weights of a gated MLP for nvfp4_linear_swiglu: W is bf16 [2F, K] with the
+ * gate projection in rows [0, F) and the up projection in rows [F, 2F); each
+ * of the two modules gets its own dynamic global scale (g_w[0] gate, g_w[1]
+ * up, device).  Codes and scales are stored with gate and up interleaved in
+ * 128-row blocks -- gate rows [128b, 128b+128) at stored rows [256b,
+ * 256b+128), up rows [128b, 128b+128) at [256b+128, 256b+256) -- so one
+ * 256-row GEMM tile holds matching gate and up columns.  codes: [2F, K/2],
+ * sf: nvfp4_sf_bytes(2F, K) bytes, ws: nvfp4_quant_workspace_bytes(2).
+ * F % 128 == 0, K % 16 == 0.
+ * Passage: gate/up are per-module-calibrated modules that serving kernels fuse
+ * into one GEMM (kipquest.com, "The abstract", "The deep dive"). */
+int nvfp4_quantize_weights_gated(const void *W, int64_t F, int64_t K, int64_t ldw,
+                                 uint8_t *codes, uint8_t *sf, float *g_w,
+                                 void *ws, size_t ws_bytes, void *stream);
+
+/* Gated-MLP up projection with the SwiGLU in the GEMM epilogue:
+ *   h[m, j] = bf16_RNE( silu(gate) * up ),  silu(v) = v / (1 + exp(-v)),
+ *   gate = fl32(acc_gate[m, j] * fl32(g_a * g_w[0])),
+ *   up   = fl32(acc_up[m, j]   * fl32(g_a * g_w[1])),
+ * with acc the fp32 block-scaled GEMM accumulators of X against the gate and
+ * up rows of a weight from nvfp4_quantize_weights_gated (X is quantized on
+ * the fly as in nvfp4_linear_fused; NVFP4_STATIC_SCALE reads its scale from the
+ * workspace the same way).  Writes h [M, F] bf16 (contiguous), then quantizes
+ * h for the next GEMM with its own dynamic scale: h_codes [M, F/2], h_sf
+ * (nvfp4_sf_bytes(M, F) bytes), *g_h (device).  The epilogue folds max|h| in
+ * as it writes h, so h is read once more, by the quantizer only.
+ * ws: nvfp4_workspace_bytes(M, 2F, K, 2) bytes.  K % 64 == 0, F % 128 == 0.
+ * Passage: the fused gate/up GEMM (kipquest.com, "The abstract"); the pages
+ * do not name the MLP activation, SiLU gating is the plain reading. */
+int nvfp4_linear_swiglu(const void *X, int64_t M, int64_t K,
+                        const uint8_t *w_codes, const uint8_t *w_sf, int64_t F, const float *g_w,
+                        void *h, uint8_t *h_codes, uint8_t *h_sf, float *g_h,
+                        unsigned flags, void *ws, size_t ws_bytes, void *stream);
+
 /* Synchronizes `stream`, then returns and clears the device status word of
  * the current device: NVFP4_OK, NVFP4_ERR_TIMEOUT or NVFP4_ERR_NONFINITE
  * (timeout wins when both are latched), or NVFP4_ERR_CUDA if the sync

@@ -84,6 +84,11 @@ struct Params {
     int32_t out_fp32;
     int32_t vec_ok;      // rows of `out` are 16-byte aligned
     uint32_t *status;
+    // gated MLP epilogue (template flag GATED): the weight is [gate F | up F]
+    // interleaved in 128-row blocks; out is h [M, F] bf16 and the largest
+    // |h| (bf16 magnitude bits) is folded into *h_amax.
+    int32_t F;
+    uint32_t *h_amax;
 };
 
 struct Smem {
@@ -166,6 +171,13 @@ __device__ __forceinline__ void store_64(const Params &p, const float *alpha, in
     }
 }
 
+// h = silu(g) * u, silu(g) = g / (1 + exp(-g)), in fp32.
+__device__ __forceinline__ float silu_mul(float g, float u)
+{
+    return __fmul_rn(__fdiv_rn(g, __fadd_rn(1.0f, expf(-g))), u);
+}
+
+template <bool GATED>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ Params p)
@@ -327,6 +339,72 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     break;
             }
         }
+    } else if (warp >= EPI_WARP0 && GATED) {
+        // ------------------------------------------- gated MLP epilogue
+        // Tile columns [0, 128) are gate rows and [128, 256) the matching up
+        // rows; each warp takes 64 of the tile's 128 h columns for its lane quarter.
+        const int q = warp & 3;
+        const int hc = (warp - EPI_WARP0) >> 2;
+        const float ga = __ldg(p.g_a);
+        const float a_gate = __fmul_rn(ga, __ldg(p.g_w));
+        const float a_up = __fmul_rn(ga, __ldg(p.g_w + 1));
+        uint32_t hmax = 0;
+        int local = 0;
+        for (int tile = blockIdx.x; tile < p.num_tiles && !sm->abort_flag; tile += gridDim.x, ++local) {
+            const int m0 = (tile % p.num_m) * BM, n0 = (tile / p.num_m) * BN;
+            const bool ok = mbar_wait_bounded(smem_u32(&sm->acc_full), local & 1, WAIT_LIMIT_NS);
+            if (!__all_sync(0xFFFFFFFFu, ok)) {
+                if (lane == 0)
+                    raise_timeout(sm, p.status);
+                break;
+            }
+            tc_fence_after();
+            const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16) + hc * 64;
+            uint32_t vg[64], vu[64];
+            tc_ld_32x32b_x64(taddr, vg);
+            tc_ld_32x32b_x64(taddr + HALF_N, vu);
+            tc_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(smem_u32(&sm->acc_empty));
+            const int row = m0 + q * 32 + lane;
+            const int col0 = (n0 >> 1) + hc * 64;  // h column
+            uint32_t pk[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                const float h0 = silu_mul(__fmul_rn(__uint_as_float(vg[2 * j]), a_gate),
+                                          __fmul_rn(__uint_as_float(vu[2 * j]), a_up));
+                const float h1 = silu_mul(__fmul_rn(__uint_as_float(vg[2 * j + 1]), a_gate),
+                                          __fmul_rn(__uint_as_float(vu[2 * j + 1]), a_up));
+                __nv_bfloat162 b = __floats2bfloat162_rn(h0, h1);
+                pk[j] = *reinterpret_cast<uint32_t *>(&b);
+            }
+            if (row < p.M && col0 < p.F) {
+                __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(p.out) + static_cast<int64_t>(row) * p.F + col0;
+                const int nval = min(64, p.F - col0);
+                if (p.vec_ok && nval == 64) {
+#pragma unroll
+                    for (int j = 0; j < 32; j += 4)
+                        *reinterpret_cast<uint4 *>(o + 2 * j) = make_uint4(pk[j], pk[j + 1], pk[j + 2], pk[j + 3]);
+#pragma unroll
+                    for (int j = 0; j < 32; ++j)
+                        hmax = vmax_mag(hmax, pk[j]);
+                } else {
+                    for (int j = 0; j < nval; ++j) {
+                        const uint32_t hb = (j & 1) ? (pk[j >> 1] >> 16) : (pk[j >> 1] & 0xFFFFu);
+                        o[j] = __ushort_as_bfloat16(static_cast<unsigned short>(hb));
+                        hmax = vmax_mag(hmax, hb);
+                    }
+                }
+            }
+        }
+        uint32_t v = hmax16(hmax);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+            v = max(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
+        if (lane == 0 && v != 0)
+            atomicMax(p.h_amax, v);
     } else if (warp >= EPI_WARP0) {
         // ------------------------------------------------------ epilogue
         const int q = warp & 3;                    // TMEM lane quarter this warp may access

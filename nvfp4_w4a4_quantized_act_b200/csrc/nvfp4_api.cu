@@ -63,7 +63,9 @@ DeviceState *device_state()
         if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess)
             return nullptr;
         d.status = static_cast<uint32_t *>(p);
-        if (cudaFuncSetAttribute(nvfp4::gemm::gemm_nvf4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (cudaFuncSetAttribute(nvfp4::gemm::gemm_nvf4_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 nvfp4::gemm::SMEM_BYTES) != cudaSuccess ||
+            cudaFuncSetAttribute(nvfp4::gemm::gemm_nvf4_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  nvfp4::gemm::SMEM_BYTES) != cudaSuccess)
             return nullptr;
         d.gemm_attr_set = true;
@@ -113,7 +115,7 @@ int launch_ok()
 // read from g_in.
 int run_quantize(DeviceState *d, const void *X, int64_t rows, int64_t K, int64_t ld, const nvfp4::SegRows &seg,
                  uint8_t *codes, uint8_t *sf, const float *g_in, float *g_out, bool dynamic, uint32_t *amax_ws,
-                 cudaStream_t stream)
+                 cudaStream_t stream, int64_t gate_up_F = 0)
 {
     const int64_t rows_pad = round_up(rows, 128);
     const int64_t groups = cdiv(K, 64);
@@ -147,8 +149,40 @@ int run_quantize(DeviceState *d, const void *X, int64_t rows, int64_t K, int64_t
     p.mode = dynamic ? 0 : 1;
     p.codes = codes;
     p.sf = sf;
+    p.gate_up_F = static_cast<int32_t>(gate_up_F);
     const int64_t threads = rows_pad * groups * 4;
     int grid = static_cast<int>(std::min<int64_t>(std::max<int64_t>(cdiv(threads, 256), 1), int64_t(d->sm_count) * 16));
+    nvfp4::quantize_kernel<<<grid, 256, 0, stream>>>(p);
+    g_launches++;
+    return launch_ok();
+}
+
+// K2 alone for a contiguous [rows, K] bf16 matrix whose amax bits are already
+// in amax_ws (one segment); writes codes, scales and g_out.
+int run_quantize_from_amax(DeviceState *d, const void *X, int64_t rows, int64_t K, const nvfp4::SegRows &seg,
+                           uint8_t *codes, uint8_t *sf, float *g_out, const uint32_t *amax_ws, cudaStream_t stream)
+{
+    const int64_t rows_pad = round_up(rows, 128);
+    const int64_t groups = cdiv(K, 64);
+    if (rows_pad * groups * 4 >= (int64_t(1) << 31))
+        return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    nvfp4::QuantParams p;
+    p.X = static_cast<const uint16_t *>(X);
+    p.ld = K;
+    p.rows = static_cast<int32_t>(rows);
+    p.K = static_cast<int32_t>(K);
+    p.rows_pad = static_cast<int32_t>(rows_pad);
+    p.groups = static_cast<int32_t>(groups);
+    p.seg = seg;
+    p.amax_bits = amax_ws;
+    p.g_in = nullptr;
+    p.g_out = g_out;
+    p.mode = 0;
+    p.codes = codes;
+    p.sf = sf;
+    p.gate_up_F = 0;
+    const int64_t threads = rows_pad * groups * 4;
+    const int grid = static_cast<int>(std::min<int64_t>(std::max<int64_t>(cdiv(threads, 256), 1), int64_t(d->sm_count) * 16));
     nvfp4::quantize_kernel<<<grid, 256, 0, stream>>>(p);
     g_launches++;
     return launch_ok();
@@ -166,9 +200,11 @@ int make_codes_map(CUtensorMap *map, const uint8_t *codes, int64_t rows, int64_t
     return r == CUDA_SUCCESS ? NVFP4_OK : NVFP4_ERR_CUDA;
 }
 
+// h_amax != nullptr selects the gated MLP epilogue (W is [gate | up]
+// interleaved in 128-row blocks, N = 2F, out = h [M, F] bf16).
 int run_gemm(DeviceState *d, const uint8_t *a_codes, const uint8_t *a_sf, const float *g_a, int64_t M, int64_t K,
              const uint8_t *w_codes, const uint8_t *w_sf, int64_t N, const nvfp4::SegRows &seg, const float *g_w,
-             void *out, unsigned flags, cudaStream_t stream)
+             void *out, unsigned flags, cudaStream_t stream, uint32_t *h_amax = nullptr)
 {
     using namespace nvfp4::gemm;
     if (M == 0 || N == 0)
@@ -200,7 +236,14 @@ int run_gemm(DeviceState *d, const uint8_t *a_codes, const uint8_t *a_sf, const 
     p.vec_ok = aligned16(out) && ((N * esz) % 16 == 0);
     p.status = d->status;
     const int grid = static_cast<int>(std::min<int64_t>(p.num_tiles, d->sm_count));
-    gemm_nvf4_kernel<<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(tmA, tmB, p);
+    if (h_amax != nullptr) {
+        p.F = static_cast<int32_t>(N / 2);
+        p.h_amax = h_amax;
+        p.vec_ok = aligned16(out) && ((p.F * 2) % 16 == 0);
+        gemm_nvf4_kernel<true><<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(tmA, tmB, p);
+    } else {
+        gemm_nvf4_kernel<false><<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(tmA, tmB, p);
+    }
     g_launches++;
     return launch_ok();
 }
@@ -218,6 +261,7 @@ int check_gemm_shape(int64_t M, int64_t N, int64_t K)
 }
 
 constexpr size_t kLinScaleOff = 256;
+constexpr size_t kLinHAmaxOff = 512;  // gated linear: max|h| word
 constexpr size_t kLinCodesOff = 1024;
 
 size_t linear_codes_bytes(int64_t M, int64_t K) { return static_cast<size_t>(M) * static_cast<size_t>(K / 2); }
@@ -466,6 +510,7 @@ int nvfp4_swiglu_quantize(const void *gate_up, int64_t M, int64_t F, int64_t ld,
     p.mode = 0;
     p.codes = codes;
     p.sf = sf;
+    p.gate_up_F = 0;
     const int64_t threads = rows_pad * groups * 4;
     const int grid = static_cast<int>(std::min<int64_t>(std::max<int64_t>(cdiv(threads, 256), 1), int64_t(d->sm_count) * 16));
     nvfp4::quantize_kernel<<<grid, 256, 0, s>>>(p);
@@ -601,4 +646,86 @@ extern "C" int nvfp4_linear_fused_noalloc(const void *X, int64_t M, int64_t K, c
     if (rc != NVFP4_OK)
         return rc;
     return run_gemm(d, a_codes, a_sf, g_a, M, K, w_codes, w_sf, N, seg, g_w, out, flags, s);
+}
+
+// ------------------------------------------------------ gated MLP (SwiGLU)
+
+extern "C" int nvfp4_quantize_weights_gated(const void *W, int64_t F, int64_t K, int64_t ldw, uint8_t *codes,
+                                            uint8_t *sf, float *g_w, void *ws, size_t ws_bytes, void *stream)
+{
+    if (W == nullptr || codes == nullptr || sf == nullptr || g_w == nullptr || F <= 0 || K <= 0)
+        return NVFP4_ERR_INVALID_ARG;
+    if (K % 16 != 0 || F % 128 != 0)
+        return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (ldw < K)
+        return NVFP4_ERR_INVALID_ARG;
+    if (!aligned16(W) || ldw % 8 != 0 || !aligned16(codes) || !aligned16(sf))
+        return NVFP4_ERR_MISALIGNED;
+    if (ws == nullptr || ws_bytes < nvfp4_quant_workspace_bytes(2))
+        return NVFP4_ERR_WORKSPACE;
+    DeviceState *d = device_state();
+    if (d == nullptr)
+        return NVFP4_ERR_CUDA;
+    if (!d->supported)
+        return NVFP4_ERR_NO_DEVICE;
+    nvfp4::SegRows seg;
+    const nvfp4_segment two[2] = {{0, F}, {F, 2 * F}};
+    check_segments(two, 2, 2 * F, &seg);
+    return run_quantize(d, W, 2 * F, K, ldw, seg, codes, sf, nullptr, g_w, true, static_cast<uint32_t *>(ws),
+                        static_cast<cudaStream_t>(stream), F);
+}
+
+extern "C" int nvfp4_linear_swiglu(const void *X, int64_t M, int64_t K, const uint8_t *w_codes, const uint8_t *w_sf,
+                                   int64_t F, const float *g_w, void *h, uint8_t *h_codes, uint8_t *h_sf, float *g_h,
+                                   unsigned flags, void *ws, size_t ws_bytes, void *stream)
+{
+    if ((flags & ~static_cast<unsigned>(NVFP4_STATIC_SCALE)) != 0)
+        return NVFP4_ERR_INVALID_ARG;
+    int rc = check_gemm_shape(M, 2 * F, K);
+    if (rc != NVFP4_OK)
+        return rc;
+    if (F <= 0)
+        return NVFP4_ERR_INVALID_ARG;
+    if (F % 128 != 0)
+        return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (g_h == nullptr || (M > 0 && (X == nullptr || w_codes == nullptr || w_sf == nullptr || g_w == nullptr ||
+                                     h == nullptr || h_codes == nullptr || h_sf == nullptr)))
+        return NVFP4_ERR_INVALID_ARG;
+    if (!aligned16(X) || K % 8 != 0 || !aligned16(w_codes) || !aligned16(w_sf) || !aligned16(h) ||
+        !aligned16(h_codes) || !aligned16(h_sf) || (reinterpret_cast<uintptr_t>(g_w) & 3u) ||
+        (reinterpret_cast<uintptr_t>(g_h) & 3u))
+        return NVFP4_ERR_MISALIGNED;
+    if (ws == nullptr || !aligned16(ws) || ws_bytes < nvfp4_workspace_bytes(M, 2 * F, K, 2))
+        return NVFP4_ERR_WORKSPACE;
+    DeviceState *d = device_state();
+    if (d == nullptr)
+        return NVFP4_ERR_CUDA;
+    if (!d->supported)
+        return NVFP4_ERR_NO_DEVICE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint8_t *base = static_cast<uint8_t *>(ws);
+    uint32_t *amax = reinterpret_cast<uint32_t *>(base);
+    float *g_a = reinterpret_cast<float *>(base + kLinScaleOff);
+    uint32_t *h_amax = reinterpret_cast<uint32_t *>(base + kLinHAmaxOff);
+    uint8_t *a_codes = base + kLinCodesOff;
+    uint8_t *a_sf = base + linear_sf_off(M, K);
+    nvfp4::SegRows one_seg;
+    nvfp4_segment one = {0, M};
+    check_segments(&one, 1, M, &one_seg);
+    // X -> NVFP4 (dynamic scale unless a calibrated one is supplied)
+    rc = run_quantize(d, X, M, K, K, one_seg, a_codes, a_sf, g_a, g_a, (flags & NVFP4_STATIC_SCALE) == 0, amax, s);
+    if (rc != NVFP4_OK)
+        return rc;
+    // gate/up GEMM with the SwiGLU epilogue -> h (bf16) and max|h|
+    if (cudaMemsetAsync(h_amax, 0, sizeof(uint32_t), s) != cudaSuccess)
+        return NVFP4_ERR_CUDA;
+    g_launches++;
+    nvfp4::SegRows gu;
+    const nvfp4_segment two[2] = {{0, F}, {F, 2 * F}};
+    check_segments(two, 2, 2 * F, &gu);
+    rc = run_gemm(d, a_codes, a_sf, g_a, M, K, w_codes, w_sf, 2 * F, gu, g_w, h, 0, s, h_amax);
+    if (rc != NVFP4_OK)
+        return rc;
+    // h -> NVFP4 with the dynamic scale folded in by the epilogue
+    return run_quantize_from_amax(d, h, M, F, one_seg, h_codes, h_sf, g_h, h_amax, s);
 }

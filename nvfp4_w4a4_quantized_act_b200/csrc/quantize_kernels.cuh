@@ -137,7 +137,22 @@ struct QuantParams {
     int32_t mode;
     uint8_t *codes;          // [rows, K/2]
     uint8_t *sf;             // swizzled scale tiles
+    int32_t gate_up_F;       // > 0: rows are [gate F | up F]; stored interleaved in 128-row blocks
 };
+
+// Stored row of input row r.  With a gate/up pair of F rows each, block b of
+// gate rows goes to stored rows [256 b, 256 b + 128) and block b of up rows to
+// [256 b + 128, 256 b + 256), so one 256-row GEMM tile holds matching gate
+// and up columns.
+__device__ __forceinline__ uint32_t stored_row(const QuantParams &p, uint32_t r)
+{
+    if (p.gate_up_F <= 0)
+        return r;
+    const uint32_t F = static_cast<uint32_t>(p.gate_up_F);
+    const uint32_t m = r >= F ? 1u : 0u;
+    const uint32_t i = r - m * F;
+    return (((i >> 7) << 1) + m) * 128u + (i & 127u);
+}
 
 __device__ __forceinline__ float global_scale_from_amax(uint32_t bits)
 {
@@ -246,7 +261,7 @@ __global__ void __launch_bounds__(256) quantize_kernel(const QuantParams p)
             const int sg = one_seg ? 0 : seg_of(p.seg, row);
             uint32_t packed[2];
             sbyte = quantize_block(v0, v1, s_g[sg], s_rg[sg], s_gok[sg] != 0, packed);
-            *reinterpret_cast<uint2 *>(p.codes + static_cast<int64_t>(row) * (p.K >> 1) + blk * 8) =
+            *reinterpret_cast<uint2 *>(p.codes + static_cast<int64_t>(stored_row(p, row)) * (p.K >> 1) + blk * 8) =
                 make_uint2(packed[0], packed[1]);
         }
         // four neighbouring blocks -> one 32-bit scale word, in lanes 0, 4, 8, ...
@@ -254,8 +269,9 @@ __global__ void __launch_bounds__(256) quantize_kernel(const QuantParams p)
         const uint32_t word = pair | (__shfl_down_sync(0xFFFFFFFFu, pair, 2) << 16);
         const uint32_t cg = chunk * 8u + (lane >> 2);
         if ((lane & 3) == 0 && cg < static_cast<uint32_t>(p.groups)) {
-            const uint64_t tile = static_cast<uint64_t>(row >> 7) * p.groups + cg;
-            const uint32_t rr = row & 127u;
+            const uint32_t srow = stored_row(p, row);
+            const uint64_t tile = static_cast<uint64_t>(srow >> 7) * p.groups + cg;
+            const uint32_t rr = srow & 127u;
             *reinterpret_cast<uint32_t *>(p.sf + tile * 512 + (rr & 31u) * 16 + (rr >> 5) * 4) = word;
         }
         row = nrow;

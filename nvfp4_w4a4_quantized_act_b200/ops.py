@@ -31,6 +31,7 @@ EXPORTED = [
     "nvfp4_quantize_weights", "nvfp4_quantize_act", "nvfp4_gemm_prequant", "nvfp4_linear_fused",
     "nvfp4_linear", "nvfp4_swiglu_quantize", "nvfp4_get_status", "nvfp4_status_string",
     "nvfp4_device_supported", "nvfp4_launch_count", "nvfp4_linear_fused_noalloc",
+    "nvfp4_quantize_weights_gated", "nvfp4_linear_swiglu",
 ]
 
 
@@ -76,6 +77,9 @@ def lib() -> ctypes.CDLL:
         "nvfp4_launch_count": (ctypes.c_uint64, []),
         "nvfp4_linear_fused_noalloc": (ctypes.c_int, [vp, i64, i64, u8p, u8p, i64, segp, fp, ctypes.c_int, vp,
                                                       ctypes.c_uint, vp]),
+        "nvfp4_quantize_weights_gated": (ctypes.c_int, [vp, i64, i64, i64, u8p, u8p, fp, vp, sz, vp]),
+        "nvfp4_linear_swiglu": (ctypes.c_int, [vp, i64, i64, u8p, u8p, i64, fp, vp, u8p, u8p, fp, ctypes.c_uint,
+                                               vp, sz, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -157,6 +161,7 @@ class QuantizedWeight:
     segments: list
     N: int
     K: int
+    gated: bool = False  # gate/up interleaved in 128-row blocks (nvfp4_quantize_weights_gated)
 
 
 def quantize_weights(W: torch.Tensor, segments=None, stream=None) -> QuantizedWeight:
@@ -300,3 +305,45 @@ def linear_fused_noalloc(X: torch.Tensor, w: QuantizedWeight, out=None, out_fp32
     _check(lib().nvfp4_linear_fused_noalloc(_p(X), M, K, _p(w.codes), _p(w.sf), w.N, arr, _p(w.g_w), n, _p(out),
                                             flags, _stream(stream)), "nvfp4_linear_fused_noalloc")
     return out
+
+
+def quantize_weights_gated(W: torch.Tensor, stream=None) -> QuantizedWeight:
+    """nvfp4_quantize_weights_gated: W = [gate F | up F] rows -> interleaved
+    gate/up NVFP4 weight with one global scale per module."""
+    _require_cuda(W)
+    assert W.dtype == torch.bfloat16 and W.dim() == 2 and W.stride(1) == 1 and W.shape[0] % 2 == 0
+    N, K = W.shape
+    F = N // 2
+    dev = W.device
+    codes = _empty_u8(N * K // 2, dev)
+    sf = _empty_u8(sf_bytes(N, K), dev)
+    g_w = torch.empty(2, dtype=torch.float32, device=dev)
+    ws = _empty_u8(quant_workspace_bytes(2), dev)
+    _check(lib().nvfp4_quantize_weights_gated(_p(W), F, K, W.stride(0), _p(codes), _p(sf), _p(g_w), _p(ws),
+                                              ws.numel(), _stream(stream)), "nvfp4_quantize_weights_gated")
+    return QuantizedWeight(codes[: N * K // 2].view(N, K // 2), sf, g_w, [(0, F), (F, N)], N, K, gated=True)
+
+
+def linear_swiglu(X: torch.Tensor, w: QuantizedWeight, h=None, h_codes=None, h_sf=None, g_h=None, ws=None,
+                  static_scale=False, stream=None):
+    """nvfp4_linear_swiglu -> (h bf16 [M, F], h_codes [M, F/2], h_sf, g_h)."""
+    _require_cuda(X)
+    assert w.gated and X.dtype == torch.bfloat16 and X.is_contiguous()
+    M, K = X.shape
+    F = w.N // 2
+    dev = X.device
+    if h is None:
+        h = torch.empty((M, F), dtype=torch.bfloat16, device=dev)
+    if h_codes is None:
+        h_codes = _empty_u8(M * F // 2, dev)
+    if h_sf is None:
+        h_sf = _empty_u8(sf_bytes(M, F), dev)
+    if g_h is None:
+        g_h = torch.empty(1, dtype=torch.float32, device=dev)
+    if ws is None:
+        ws = _empty_u8(workspace_bytes(M, w.N, K, 2), dev)
+    flags = NVFP4_STATIC_SCALE if static_scale else 0
+    _check(lib().nvfp4_linear_swiglu(_p(X), M, K, _p(w.codes), _p(w.sf), F, _p(w.g_w), _p(h), _p(h_codes),
+                                     _p(h_sf), _p(g_h), flags, _p(ws), ws.numel(), _stream(stream)),
+           "nvfp4_linear_swiglu")
+    return h, h_codes[: M * F // 2].view(M, F // 2), h_sf, g_h

@@ -271,3 +271,27 @@ def swiglu(gate_up_bits: np.ndarray) -> np.ndarray:
     h = np.zeros((rows, F), dtype=np.uint16)
     _L().oracle_swiglu(_ptr(x), rows, F, F2, _ptr(h))
     return h
+
+
+# ------------------------------------------------------ gated MLP (fused)
+
+def gated_stored_row(r: int, F: int) -> int:
+    """Row at which the gated weight layout stores input row r of a [gate F |
+    up F] weight: 128-row blocks alternate gate, up, gate, up, ..."""
+    module, i = divmod(r, F)
+    block, within = divmod(i, 128)
+    return (2 * block + module) * 128 + within
+
+
+def interleave_gate_up(rows_data: np.ndarray, F: int) -> np.ndarray:
+    """Reorder the rows of a [2F, ...] array into the gated storage order."""
+    out = np.empty_like(rows_data)
+    for r in range(2 * F):
+        out[gated_stored_row(r, F)] = rows_data[r]
+    return out
+
+
+def silu_mul(g: np.ndarray, u: np.ndarray) -> np.ndarray:
+    """silu(g) * u = g / (1 + exp(-g)) * u, in fp64."""
+    g = np.asarray(g, dtype=np.float64)
+    return g / (1.0 + np.exp(-g)) * np.asarray(u, dtype=np.float64)

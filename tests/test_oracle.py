@@ -402,3 +402,27 @@ def test_swiglu_against_torch_float64():
     ulp = np.exp2(np.floor(np.log2(np.maximum(np.abs(ref), 1e-38))) - 7)
     assert np.all(np.abs(hv - ref) <= 0.5 * ulp * (1 + 1e-9))
     assert np.all(hv[gu[:, :32].float().numpy() == 0] == 0)
+
+
+# ------------------------------------------------- gated MLP weight layout
+
+def test_gated_layout_alternates_gate_and_up_blocks():
+    F = 384
+    rows = [oracle.gated_stored_row(r, F) for r in range(2 * F)]
+    assert sorted(rows) == list(range(2 * F))                     # a permutation
+    assert rows[0] == 0 and rows[127] == 127 and rows[128] == 256  # gate blocks at even 128-row slots
+    assert rows[F] == 128 and rows[F + 127] == 255 and rows[2 * F - 1] == 2 * F - 1  # up blocks at odd slots
+    data = np.arange(2 * F)
+    inter = oracle.interleave_gate_up(data, F)
+    for t in range(2 * F // 256):
+        assert np.array_equal(inter[256 * t: 256 * t + 128], data[128 * t: 128 * t + 128])
+        assert np.array_equal(inter[256 * t + 128: 256 * t + 256], data[F + 128 * t: F + 128 * t + 128])
+
+
+def test_silu_mul_against_torch():
+    rng = np.random.default_rng(17)
+    g = rng.standard_normal(1000) * 8
+    u = rng.standard_normal(1000)
+    ref = (torch.nn.functional.silu(torch.from_numpy(g)) * torch.from_numpy(u)).numpy()
+    assert np.allclose(oracle.silu_mul(g, u), ref, rtol=1e-14, atol=1e-300)
+    assert oracle.silu_mul(0.0, 3.0) == 0.0
