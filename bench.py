@@ -7,8 +7,9 @@ scale per module (4 GEMMs a layer, 256 a step):
 
   GDN layer       in_proj [qkv 8192 | z 6144 | b 48 | a 48] <- X (5120)
                   out      5120 <- Y (6144)
-                  gate_up [gate 17408 | up 17408] <- X2 (5120)
-                  down     5120 <- h = silu(gate) * up (17408)
+                  gate_up [gate 17408 | up 17408] <- X2 (5120), SwiGLU in the
+                           epilogue: h = silu(gate) * up (17408)
+                  down     5120 <- h
   attention layer qkv [q+gate 12288 | k 1024 | v 1024] <- X, o 5120 <- Y,
                   gate_up, down as above
 
@@ -45,6 +46,19 @@ METRIC = "NVFP4 W4A4 linear TFLOPS (quant+GEMM) at prefill shapes; % of FP4 & HB
 WORKLOAD = "496-linear hybrid stack (48 GDN + 16 attention layers, hidden 5120, MLP 17408), one 8192-token prefill chunk"
 FP4_PER_BF16 = 4.0  # dense FP4 : dense BF16 tensor throughput on B200 (9 : 2.25 PFLOP/s nominal)
 FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# DRAM bytes (read + write) per GEMM launch, mean over the four GEMM launches of
+# one layer, from one ncu capture of this kernel source (profiles/
+# gemm_nvf4_kernel_layer_8192tok.md gives the command).  Reported only while
+# the kernel source still has the captured hash.
+GEMM_TRAFFIC = {"source_sha256_12": "cb4df766954e", "bytes_per_launch": 266.044e6}
+GEMM_SOURCE = os.path.join(ROOT, "nvfp4_w4a4_quantized_act_b200", "csrc", "gemm_kernel.cuh")
+
+
+def gemm_traffic():
+    import hashlib
+    with open(GEMM_SOURCE, "rb") as f:
+        h = hashlib.sha256(f.read()).hexdigest()[:12]
+    return GEMM_TRAFFIC["bytes_per_launch"] if h == GEMM_TRAFFIC["source_sha256_12"] else None
 
 
 def parse_args():
@@ -151,7 +165,10 @@ class Stack:
                          for j, m in enumerate(lin.modules)]
                 W = torch.cat(parts, 0) if len(parts) > 1 else parts[0]
                 del parts
-                qs.append(ops.quantize_weights(W, lin.segments))
+                if lin.name == "gate_up":
+                    qs.append(ops.quantize_weights_gated(W))
+                else:
+                    qs.append(ops.quantize_weights(W, lin.segments))
                 del W
             self.weights.append(qs)
         torch.cuda.synchronize()
@@ -162,13 +179,15 @@ class Stack:
         self.outs = {}
         for _, lins in self.layers[:4]:
             for lin in lins:
-                self.outs.setdefault((lin.name, lin.N), torch.empty((TOKENS, lin.N), dtype=torch.bfloat16,
-                                                                     device=device))
+                if lin.name != "gate_up":
+                    self.outs.setdefault((lin.name, lin.N), torch.empty((TOKENS, lin.N), dtype=torch.bfloat16,
+                                                                         device=device))
         maxK = max(lin.K for _, lins in self.layers for lin in lins)
         self.a_codes = torch.empty(TOKENS * maxK // 2, dtype=torch.uint8, device=device)
         self.a_sf = torch.empty(ops.sf_bytes(TOKENS, maxK), dtype=torch.uint8, device=device)
         self.g_a = torch.empty(1, dtype=torch.float32, device=device)
         self.qws = torch.empty(ops.quant_workspace_bytes(1), dtype=torch.uint8, device=device)
+        self.hws = torch.empty(ops.quant_workspace_bytes(1), dtype=torch.uint8, device=device)
         self.h = torch.empty((TOKENS, 17408), dtype=torch.bfloat16, device=device)
         self.lin_ws = torch.empty(ops.workspace_bytes(TOKENS, 0, maxK), dtype=torch.uint8, device=device)
         self.flops = stack_flops(self.layers)
@@ -182,45 +201,46 @@ class Stack:
         return self.X
 
     def step_split(self, gemm_events=None):
-        """One step through nvfp4_quantize_act / nvfp4_swiglu_quantize /
-        nvfp4_gemm_prequant, with CUDA events around each GEMM launch."""
+        """One step through nvfp4_quantize_act / nvfp4_gemm_prequant(_swiglu),
+        with CUDA events around each GEMM launch."""
         ops = self.ops
         k = 0
         for qs, (_, lins) in zip(self.weights, self.layers):
             for lin, qw in zip(lins, qs):
-                out = self.outs[(lin.name, lin.N)]
                 if lin.name == "down":
-                    gu = self.outs[("gate_up", 34816)]
-                    _, hc, hsf, gh = ops.swiglu_quantize(gu, h=self.h, codes=self.a_codes, sf=self.a_sf,
-                                                         g_h=self.g_a, ws=self.qws)
-                    ac, asf = hc, hsf
+                    # h was written by the gated epilogue, its max|h| is in hws
+                    ac, asf, _ = ops.quantize_act(self.h, g_a=self.g_a, codes=self.a_codes, sf=self.a_sf,
+                                                  ws=self.hws, amax_given=True)
                 else:
                     ac, asf, _ = ops.quantize_act(self._input(lin), g_a=self.g_a, codes=self.a_codes, sf=self.a_sf,
                                                   ws=self.qws)
                 if gemm_events is not None:
                     gemm_events[k][0].record()
-                ops.gemm_prequant(ac, asf, self.g_a, TOKENS, lin.K, qw, out=out)
+                if lin.name == "gate_up":
+                    ops.gemm_prequant_swiglu(ac, asf, self.g_a, TOKENS, lin.K, qw, h=self.h, ws=self.hws)
+                else:
+                    ops.gemm_prequant(ac, asf, self.g_a, TOKENS, lin.K, qw, out=self.outs[(lin.name, lin.N)])
                 if gemm_events is not None:
                     gemm_events[k][1].record()
                 k += 1
 
     def step_public(self):
-        """One step through the user-facing calls (nvfp4_linear_fused for
-        every fused GEMM, nvfp4_swiglu_quantize + nvfp4_gemm_prequant for the
-        down projection)."""
+        """One step through the user-facing calls (nvfp4_linear_fused for the
+        fused projections, nvfp4_linear_swiglu for gate/up + SwiGLU, and
+        nvfp4_gemm_prequant on the quantized h for the down projection)."""
         ops = self.ops
         last = None
         for qs, (_, lins) in zip(self.weights, self.layers):
             for lin, qw in zip(lins, qs):
-                out = self.outs[(lin.name, lin.N)]
-                if lin.name == "down":
-                    gu = self.outs[("gate_up", 34816)]
-                    _, hc, hsf, gh = ops.swiglu_quantize(gu, h=self.h, codes=self.a_codes, sf=self.a_sf,
-                                                         g_h=self.g_a, ws=self.qws)
+                if lin.name == "gate_up":
+                    _, hc, hsf, gh = ops.linear_swiglu(self.X2, qw, h=self.h, h_codes=self.a_codes, h_sf=self.a_sf,
+                                                       g_h=self.g_a, ws=self.lin_ws)
+                elif lin.name == "down":
+                    out = self.outs[(lin.name, lin.N)]
                     ops.gemm_prequant(hc, hsf, gh, TOKENS, lin.K, qw, out=out)
+                    last = out
                 else:
-                    ops.linear_fused(self._input(lin), qw, out=out, ws=self.lin_ws)
-                last = out
+                    ops.linear_fused(self._input(lin), qw, out=self.outs[(lin.name, lin.N)], ws=self.lin_ws)
         return last
 
 
@@ -334,13 +354,15 @@ def bench_gpu(args, rank, world, local):
             "parallelism": f"replicas x{world} (no collectives)",
         },
         "roofline": {
-            "kernel": "gemm_nvf4_kernel (tcgen05 block-scaled FP4 GEMM + per-module scale epilogue)",
+            "kernel": "gemm_nvf4_kernel (tcgen05 block-scaled FP4 GEMM; per-module-scale or SwiGLU epilogue)",
             "bound": "tensor",
             "achieved": round(gemm_tflops, 1),
             "peak": round(fp4_peak, 1),
             "unit": "TFLOP/s",
             "frac": round(gemm_tflops / fp4_peak, 4),
-            "traffic": None,
+            "traffic": gemm_traffic(),
+            "traffic_unit": "bytes per launch (DRAM read+write, ncu, mean of one layer's 4 GEMMs)",
+            "algorithmic_bytes_per_launch": round(gemm_alg_bytes(stack), 0),
             "peak_basis": f"{pk_kind} bf16 sustained {pk['bf16_tflops_sustained']} TF/s x {FP4_PER_BF16} "
                           "(nominal dense FP4:BF16 ratio)",
             "frac_of_datasheet_9pf": round(gemm_tflops / 9000.0, 4),
@@ -353,6 +375,18 @@ def bench_gpu(args, rank, world, local):
     if e2e is not None:
         res["e2e"] = e2e
     return res
+
+
+def gemm_alg_bytes(stack) -> float:
+    """Mean algorithmic bytes per GEMM launch over the step: codes (K/2 per
+    row) and scales (K/16 per row) of both operands plus the bf16 output."""
+    tot, n = 0.0, 0
+    for _, lins in stack.layers:
+        for lin in lins:
+            out_cols = lin.N // 2 if lin.name == "gate_up" else lin.N
+            tot += (TOKENS + lin.N) * lin.K * (0.5 + 1 / 16) + TOKENS * out_cols * 2
+            n += 1
+    return tot / n
 
 
 def quantize_roofline(stack, pk, pk_kind):
@@ -410,7 +444,7 @@ def bench_e2e(stack, args, world):
     ms = max_over_ranks(s.elapsed_time(e), world) / args.steps
     return {"value": round(stack.flops * world / (ms * 1e-3) / 1e12, 2), "unit": "TFLOPS",
             "ms_per_step": round(ms, 3), "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-            "api": "nvfp4_linear_fused / nvfp4_swiglu_quantize / nvfp4_gemm_prequant"}
+            "api": "nvfp4_linear_fused / nvfp4_linear_swiglu / nvfp4_gemm_prequant"}
 
 
 # ------------------------------------------------------ CPU oracle legs

@@ -83,6 +83,9 @@ typedef struct {
 /* Flags. */
 #define NVFP4_STATIC_SCALE 1u /* activation global scale is an input (calibrated), not computed */
 #define NVFP4_OUT_FP32 2u     /* GEMM output is fp32 instead of bf16 */
+#define NVFP4_AMAX_GIVEN 4u   /* nvfp4_quantize_act: the first word of ws already holds max|X|
+                               * (bf16 magnitude bits, as nvfp4_gemm_prequant_swiglu leaves
+                               * it); skip the amax pass */
 
 /* Bytes of the swizzled scale-factor buffer for a [rows, K] matrix:
  * ceil(rows/128)*128 * ceil(K/64)*4.  Returns 0 for invalid sizes. */
@@ -180,6 +183,16 @@ int nvfp4_swiglu_quantize(const void *gate_up, int64_t M, int64_t F, int64_t ld,
 int nvfp4_quantize_weights_gated(const void *W, int64_t F, int64_t K, int64_t ldw,
                                  uint8_t *codes, uint8_t *sf, float *g_w,
                                  void *ws, size_t ws_bytes, void *stream);
+
+/* The gated GEMM of nvfp4_linear_swiglu on already-quantized activations
+ * (a_codes/a_sf/g_a as from nvfp4_quantize_act): writes h [M, F] bf16 and
+ * leaves max|h| (bf16 magnitude bits) in the first word of ws (>= 256 bytes),
+ * ready for nvfp4_quantize_act(h, ..., NVFP4_AMAX_GIVEN, ws, ...).
+ * K % 64 == 0, F % 128 == 0. */
+int nvfp4_gemm_prequant_swiglu(const uint8_t *a_codes, const uint8_t *a_sf, const float *g_a,
+                               int64_t M, int64_t K, const uint8_t *w_codes, const uint8_t *w_sf,
+                               int64_t F, const float *g_w, void *h, void *ws, size_t ws_bytes,
+                               void *stream);
 
 /* Gated-MLP up projection with the SwiGLU in the GEMM epilogue:
  *   h[m, j] = bf16_RNE( silu(gate) * up ),  silu(v) = v / (1 + exp(-v)),

@@ -89,7 +89,23 @@ struct Params {
     // |h| (bf16 magnitude bits) is folded into *h_amax.
     int32_t F;
     uint32_t *h_amax;
+    // Tile order: consecutive tiles (run at the same time by neighbouring
+    // CTAs) share their A block when n_fastest, else their W block, so the
+    // operand re-read for every tile column / row is the smaller one and stays
+    // in L2.
+    int32_t n_fastest;
 };
+
+__device__ __forceinline__ void tile_coords(const Params &p, int tile, int &m_blk, int &n_blk)
+{
+    if (p.n_fastest) {
+        n_blk = tile % p.num_n;
+        m_blk = tile / p.num_n;
+    } else {
+        m_blk = tile % p.num_m;
+        n_blk = tile / p.num_m;
+    }
+}
 
 struct Smem {
     uint64_t full[STAGES];
@@ -225,7 +241,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             int stage = 0;
             uint32_t phase = 0;
             for (int tile = blockIdx.x; tile < p.num_tiles && !sm->abort_flag; tile += gridDim.x) {
-                const int m_blk = tile % p.num_m, n_blk = tile / p.num_m;
+                int m_blk, n_blk;
+                tile_coords(p, tile, m_blk, n_blk);
                 const int m0 = m_blk * BM, n0 = n_blk * BN;
                 const int rb0 = n0 >> 7;  // first 128-row scale tile of W
                 const int nb_tiles = (rb0 + 1 < p.n_row_tiles) ? 2 : 1;
@@ -351,7 +368,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         uint32_t hmax = 0;
         int local = 0;
         for (int tile = blockIdx.x; tile < p.num_tiles && !sm->abort_flag; tile += gridDim.x, ++local) {
-            const int m0 = (tile % p.num_m) * BM, n0 = (tile / p.num_m) * BN;
+            int m_blk, n_blk;
+            tile_coords(p, tile, m_blk, n_blk);
+            const int m0 = m_blk * BM, n0 = n_blk * BN;
             const bool ok = mbar_wait_bounded(smem_u32(&sm->acc_full), local & 1, WAIT_LIMIT_NS);
             if (!__all_sync(0xFFFFFFFFu, ok)) {
                 if (lane == 0)
@@ -413,7 +432,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const float ga = __ldg(p.g_a);
         int local = 0;
         for (int tile = blockIdx.x; tile < p.num_tiles && !sm->abort_flag; tile += gridDim.x, ++local) {
-            const int m0 = (tile % p.num_m) * BM, n0 = (tile / p.num_m) * BN;
+            int m_blk, n_blk;
+            tile_coords(p, tile, m_blk, n_blk);
+            const int m0 = m_blk * BM, n0 = n_blk * BN;
             __syncwarp();  // this warp's reads of the previous tile's alpha are done
 #pragma unroll
             for (int j = 0; j < HALF_N / 32; ++j)

@@ -159,7 +159,7 @@ int run_quantize(DeviceState *d, const void *X, int64_t rows, int64_t K, int64_t
 
 // K2 alone for a contiguous [rows, K] bf16 matrix whose amax bits are already
 // in amax_ws (one segment); writes codes, scales and g_out.
-int run_quantize_from_amax(DeviceState *d, const void *X, int64_t rows, int64_t K, const nvfp4::SegRows &seg,
+int run_quantize_from_amax(DeviceState *d, const void *X, int64_t rows, int64_t K, int64_t ld, const nvfp4::SegRows &seg,
                            uint8_t *codes, uint8_t *sf, float *g_out, const uint32_t *amax_ws, cudaStream_t stream)
 {
     const int64_t rows_pad = round_up(rows, 128);
@@ -168,7 +168,7 @@ int run_quantize_from_amax(DeviceState *d, const void *X, int64_t rows, int64_t 
         return NVFP4_ERR_UNSUPPORTED_SHAPE;
     nvfp4::QuantParams p;
     p.X = static_cast<const uint16_t *>(X);
-    p.ld = K;
+    p.ld = ld;
     p.rows = static_cast<int32_t>(rows);
     p.K = static_cast<int32_t>(K);
     p.rows_pad = static_cast<int32_t>(rows_pad);
@@ -235,6 +235,8 @@ int run_gemm(DeviceState *d, const uint8_t *a_codes, const uint8_t *a_sf, const 
     const int64_t esz = p.out_fp32 ? 4 : 2;
     p.vec_ok = aligned16(out) && ((N * esz) % 16 == 0);
     p.status = d->status;
+    // re-stream the smaller operand: A is M x K/2 bytes of codes, W is N x K/2
+    p.n_fastest = (M > N) ? 1 : 0;
     const int grid = static_cast<int>(std::min<int64_t>(p.num_tiles, d->sm_count));
     if (h_amax != nullptr) {
         p.F = static_cast<int32_t>(N / 2);
@@ -333,7 +335,8 @@ int nvfp4_quantize_act(const void *X, int64_t M, int64_t K, int64_t ldx, uint8_t
 {
     if (g_a == nullptr || M < 0 || K <= 0 || (M > 0 && (X == nullptr || codes == nullptr || sf == nullptr)))
         return NVFP4_ERR_INVALID_ARG;
-    if ((flags & ~(NVFP4_STATIC_SCALE | NVFP4_OUT_FP32)) != 0)
+    if ((flags & ~(NVFP4_STATIC_SCALE | NVFP4_OUT_FP32 | NVFP4_AMAX_GIVEN)) != 0 ||
+        ((flags & NVFP4_STATIC_SCALE) && (flags & NVFP4_AMAX_GIVEN)))
         return NVFP4_ERR_INVALID_ARG;
     if (K % 16 != 0)
         return NVFP4_ERR_UNSUPPORTED_SHAPE;
@@ -353,6 +356,9 @@ int nvfp4_quantize_act(const void *X, int64_t M, int64_t K, int64_t ldx, uint8_t
     nvfp4::SegRows seg;
     nvfp4_segment one = {0, M};
     check_segments(&one, 1, M, &seg);
+    if (flags & NVFP4_AMAX_GIVEN)
+        return run_quantize_from_amax(d, X, M, K, ldx, seg, codes, sf, g_a, static_cast<const uint32_t *>(ws),
+                                      static_cast<cudaStream_t>(stream));
     return run_quantize(d, X, M, K, ldx, seg, codes, sf, g_a, g_a, dynamic, static_cast<uint32_t *>(ws),
                         static_cast<cudaStream_t>(stream));
 }
@@ -675,6 +681,41 @@ extern "C" int nvfp4_quantize_weights_gated(const void *W, int64_t F, int64_t K,
                         static_cast<cudaStream_t>(stream), F);
 }
 
+extern "C" int nvfp4_gemm_prequant_swiglu(const uint8_t *a_codes, const uint8_t *a_sf, const float *g_a, int64_t M,
+                                          int64_t K, const uint8_t *w_codes, const uint8_t *w_sf, int64_t F,
+                                          const float *g_w, void *h, void *ws, size_t ws_bytes, void *stream)
+{
+    int rc = check_gemm_shape(M, 2 * F, K);
+    if (rc != NVFP4_OK)
+        return rc;
+    if (F <= 0)
+        return NVFP4_ERR_INVALID_ARG;
+    if (F % 128 != 0)
+        return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (ws == nullptr || ws_bytes < nvfp4_quant_workspace_bytes(1))
+        return NVFP4_ERR_WORKSPACE;
+    if (M > 0 && (a_codes == nullptr || a_sf == nullptr || g_a == nullptr || w_codes == nullptr ||
+                  w_sf == nullptr || g_w == nullptr || h == nullptr))
+        return NVFP4_ERR_INVALID_ARG;
+    if (!aligned16(a_codes) || !aligned16(a_sf) || !aligned16(w_codes) || !aligned16(w_sf) || !aligned16(h) ||
+        !aligned16(ws) || (reinterpret_cast<uintptr_t>(g_a) & 3u) || (reinterpret_cast<uintptr_t>(g_w) & 3u))
+        return NVFP4_ERR_MISALIGNED;
+    DeviceState *d = device_state();
+    if (d == nullptr)
+        return NVFP4_ERR_CUDA;
+    if (!d->supported)
+        return NVFP4_ERR_NO_DEVICE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint32_t *h_amax = static_cast<uint32_t *>(ws);
+    if (cudaMemsetAsync(h_amax, 0, sizeof(uint32_t), s) != cudaSuccess)
+        return NVFP4_ERR_CUDA;
+    g_launches++;
+    nvfp4::SegRows gu;
+    const nvfp4_segment two[2] = {{0, F}, {F, 2 * F}};
+    check_segments(two, 2, 2 * F, &gu);
+    return run_gemm(d, a_codes, a_sf, g_a, M, K, w_codes, w_sf, 2 * F, gu, g_w, h, 0, s, h_amax);
+}
+
 extern "C" int nvfp4_linear_swiglu(const void *X, int64_t M, int64_t K, const uint8_t *w_codes, const uint8_t *w_sf,
                                    int64_t F, const float *g_w, void *h, uint8_t *h_codes, uint8_t *h_sf, float *g_h,
                                    unsigned flags, void *ws, size_t ws_bytes, void *stream)
@@ -727,5 +768,5 @@ extern "C" int nvfp4_linear_swiglu(const void *X, int64_t M, int64_t K, const ui
     if (rc != NVFP4_OK)
         return rc;
     // h -> NVFP4 with the dynamic scale folded in by the epilogue
-    return run_quantize_from_amax(d, h, M, F, one_seg, h_codes, h_sf, g_h, h_amax, s);
+    return run_quantize_from_amax(d, h, M, F, F, one_seg, h_codes, h_sf, g_h, h_amax, s);
 }

@@ -18,6 +18,7 @@ LIB_PATH = os.path.join(_PKG, "libnvfp4.so")
 
 NVFP4_STATIC_SCALE = 1
 NVFP4_OUT_FP32 = 2
+NVFP4_AMAX_GIVEN = 4
 MAX_SEGMENTS = 16
 
 STATUS_NAMES = {
@@ -31,7 +32,7 @@ EXPORTED = [
     "nvfp4_quantize_weights", "nvfp4_quantize_act", "nvfp4_gemm_prequant", "nvfp4_linear_fused",
     "nvfp4_linear", "nvfp4_swiglu_quantize", "nvfp4_get_status", "nvfp4_status_string",
     "nvfp4_device_supported", "nvfp4_launch_count", "nvfp4_linear_fused_noalloc",
-    "nvfp4_quantize_weights_gated", "nvfp4_linear_swiglu",
+    "nvfp4_quantize_weights_gated", "nvfp4_linear_swiglu", "nvfp4_gemm_prequant_swiglu",
 ]
 
 
@@ -80,6 +81,7 @@ def lib() -> ctypes.CDLL:
         "nvfp4_quantize_weights_gated": (ctypes.c_int, [vp, i64, i64, i64, u8p, u8p, fp, vp, sz, vp]),
         "nvfp4_linear_swiglu": (ctypes.c_int, [vp, i64, i64, u8p, u8p, i64, fp, vp, u8p, u8p, fp, ctypes.c_uint,
                                                vp, sz, vp]),
+        "nvfp4_gemm_prequant_swiglu": (ctypes.c_int, [u8p, u8p, fp, i64, i64, u8p, u8p, i64, fp, vp, vp, sz, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -182,7 +184,7 @@ def quantize_weights(W: torch.Tensor, segments=None, stream=None) -> QuantizedWe
 
 
 def quantize_act(X: torch.Tensor, g_a: torch.Tensor | None = None, static_scale: bool = False, codes=None,
-                 sf=None, ws=None, stream=None):
+                 sf=None, ws=None, stream=None, amax_given: bool = False):
     """nvfp4_quantize_act -> (codes [M, K/2] u8, swizzled sf u8, g_a fp32[1])."""
     _require_cuda(X)
     assert X.dtype == torch.bfloat16 and X.dim() == 2 and X.stride(1) == 1
@@ -197,7 +199,7 @@ def quantize_act(X: torch.Tensor, g_a: torch.Tensor | None = None, static_scale:
         g_a = torch.empty(1, dtype=torch.float32, device=dev)
     if ws is None:
         ws = _empty_u8(quant_workspace_bytes(1), dev)
-    flags = NVFP4_STATIC_SCALE if static_scale else 0
+    flags = (NVFP4_STATIC_SCALE if static_scale else 0) | (NVFP4_AMAX_GIVEN if amax_given else 0)
     _check(lib().nvfp4_quantize_act(_p(X), M, K, X.stride(0), _p(codes), _p(sf), _p(g_a), flags, _p(ws),
                                     ws.numel(), _stream(stream)), "nvfp4_quantize_act")
     return codes[: M * K // 2].view(M, K // 2), sf, g_a
@@ -347,3 +349,18 @@ def linear_swiglu(X: torch.Tensor, w: QuantizedWeight, h=None, h_codes=None, h_s
                                      _p(h_sf), _p(g_h), flags, _p(ws), ws.numel(), _stream(stream)),
            "nvfp4_linear_swiglu")
     return h, h_codes[: M * F // 2].view(M, F // 2), h_sf, g_h
+
+
+def gemm_prequant_swiglu(a_codes, a_sf, g_a, M: int, K: int, w: QuantizedWeight, h=None, ws=None, stream=None):
+    """nvfp4_gemm_prequant_swiglu -> (h bf16 [M, F], ws holding max|h|)."""
+    _require_cuda(a_codes, a_sf, g_a)
+    assert w.gated
+    F = w.N // 2
+    if h is None:
+        h = torch.empty((M, F), dtype=torch.bfloat16, device=a_codes.device)
+    if ws is None:
+        ws = _empty_u8(quant_workspace_bytes(1), a_codes.device)
+    _check(lib().nvfp4_gemm_prequant_swiglu(_p(a_codes), _p(a_sf), _p(g_a), M, K, _p(w.codes), _p(w.sf), F,
+                                            _p(w.g_w), _p(h), _p(ws), ws.numel(), _stream(stream)),
+           "nvfp4_gemm_prequant_swiglu")
+    return h, ws

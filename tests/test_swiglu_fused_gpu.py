@@ -88,3 +88,18 @@ def test_linear_swiglu_prefill_mlp_full_size():
     rows = np.unique(np.concatenate([rng.integers(0, M, 24), [0, M - 1]]))
     cols = np.unique(np.concatenate([rng.integers(0, F, 96), np.arange(F - 130, F)]))
     _check(M, K, F, X, W, rows, cols)
+
+
+def test_split_calls_equal_linear_swiglu():
+    """nvfp4_quantize_act + nvfp4_gemm_prequant_swiglu + nvfp4_quantize_act
+    (NVFP4_AMAX_GIVEN) is nvfp4_linear_swiglu, bit for bit."""
+    M, K, F = 130, 256, 256
+    X = wl.activation_normal(M, K, 60).to(DEV)
+    qw = ops.quantize_weights_gated(_gate_up(F, K, 61).to(DEV))
+    h1, c1, s1, g1 = ops.linear_swiglu(X, qw)
+    ac, asf, ga = ops.quantize_act(X)
+    h2, ws = ops.gemm_prequant_swiglu(ac, asf, ga, M, K, qw)
+    c2, s2, g2 = ops.quantize_act(h2, ws=ws, amax_given=True)
+    assert ops.get_status() == 0
+    assert torch.equal(h1, h2) and torch.equal(g1, g2)
+    assert torch.equal(c1, c2) and torch.equal(s1[: ops.sf_bytes(M, F)], s2[: ops.sf_bytes(M, F)])
