@@ -277,6 +277,12 @@ def max_over_ranks(x: float, world: int) -> float:
     return float(t.item())
 
 
+def aggregate_throughput(flops_per_rank_step: float, world: int, ms_per_step: float) -> float:
+    """TFLOPS of the whole job: the work of every rank over the slowest
+    rank's step time."""
+    return flops_per_rank_step * world / (ms_per_step * 1e-3) / 1e12
+
+
 def bench_gpu(args, rank, world, local):
     from nvfp4_w4a4_quantized_act_b200 import build as nbuild
     from nvfp4_w4a4_quantized_act_b200 import ops
@@ -320,7 +326,7 @@ def bench_gpu(args, rank, world, local):
         raise RuntimeError(f"device status {status} after the timed region")
 
     ms_per_step = elapsed_ms / args.steps
-    value = stack.flops * world / (ms_per_step * 1e-3) / 1e12
+    value = aggregate_throughput(stack.flops, world, ms_per_step)
     gemm_tflops = sum(stack.gemm_flops) / (sum(gemm_ms) * 1e-3) / 1e12
     pk, pk_kind = peaks()
     fp4_peak = pk["bf16_tflops_sustained"] * FP4_PER_BF16
@@ -442,7 +448,7 @@ def bench_e2e(stack, args, world):
     torch.cuda.synchronize()
     barrier(world)
     ms = max_over_ranks(s.elapsed_time(e), world) / args.steps
-    return {"value": round(stack.flops * world / (ms * 1e-3) / 1e12, 2), "unit": "TFLOPS",
+    return {"value": round(aggregate_throughput(stack.flops, world, ms), 2), "unit": "TFLOPS",
             "ms_per_step": round(ms, 3), "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
             "api": "nvfp4_linear_fused / nvfp4_linear_swiglu / nvfp4_gemm_prequant"}
 

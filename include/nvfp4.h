@@ -83,6 +83,10 @@ typedef struct {
 /* Flags. */
 #define NVFP4_STATIC_SCALE 1u /* activation global scale is an input (calibrated), not computed */
 #define NVFP4_OUT_FP32 2u     /* GEMM output is fp32 instead of bf16 */
+#define NVFP4_DEBUG_INJECT_STALL (1u << 30) /* nvfp4_gemm_prequant only: the kernel's loads are
+                               * skipped so its bounded waits run out (20 ms) and it
+                               * unwinds, latching NVFP4_ERR_TIMEOUT; outputs are not
+                               * written.  Exercises the failure path without a hang. */
 #define NVFP4_AMAX_GIVEN 4u   /* nvfp4_quantize_act: the first word of ws already holds max|X|
                                * (bf16 magnitude bits, as nvfp4_gemm_prequant_swiglu leaves
                                * it); skip the amax pass */

@@ -59,7 +59,7 @@ constexpr int NUM_THREADS = 384;
 constexpr int EPI_WARP0 = 4;
 constexpr int EPI_THREADS = 256;
 constexpr uint32_t SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 5120 /*barriers, alpha*/;
-constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;           // 2 s per wait
+constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;           // default bound of every wait: 2 s
 
 static_assert(SF_COL0 + STAGES * SF_BUF_COLS <= TMEM_COLS, "TMEM budget");
 static_assert(STAGE_BYTES % 1024 == 0, "stage alignment for the 128-byte swizzle");
@@ -94,6 +94,10 @@ struct Params {
     // operand re-read for every tile column / row is the smaller one and stays
     // in L2.
     int32_t n_fastest;
+    // Failure-path check: the producer issues nothing, so every consumer's
+    // bounded wait runs out after wait_limit_ns and the kernel unwinds.
+    int32_t inject_stall;
+    uint64_t wait_limit_ns;
 };
 
 __device__ __forceinline__ void tile_coords(const Params &p, int tile, int &m_blk, int &n_blk)
@@ -237,7 +241,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
     if (warp == 0) {
         // ------------------------------------------------------ producer
-        if (lane == 0) {
+        if (lane == 0 && !p.inject_stall) {
             int stage = 0;
             uint32_t phase = 0;
             for (int tile = blockIdx.x; tile < p.num_tiles && !sm->abort_flag; tile += gridDim.x) {
@@ -247,7 +251,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 const int rb0 = n0 >> 7;  // first 128-row scale tile of W
                 const int nb_tiles = (rb0 + 1 < p.n_row_tiles) ? 2 : 1;
                 for (int kt = 0; kt < p.kt_total; ++kt) {
-                    if (!mbar_wait_bounded(smem_u32(&sm->empty[stage]), phase ^ 1u, WAIT_LIMIT_NS)) {
+                    if (!mbar_wait_bounded(smem_u32(&sm->empty[stage]), phase ^ 1u, p.wait_limit_ns)) {
                         raise_timeout(sm, p.status);
                         break;
                     }
@@ -278,15 +282,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             uint32_t phase = 0;
             int local = 0;
             for (int tile = blockIdx.x; tile < p.num_tiles && !sm->abort_flag; tile += gridDim.x, ++local) {
-                if (!mbar_wait_bounded(smem_u32(&sm->acc_empty), (local & 1) ^ 1u, WAIT_LIMIT_NS)) {
+                if (!mbar_wait_bounded(smem_u32(&sm->acc_empty), (local & 1) ^ 1u, p.wait_limit_ns)) {
                     raise_timeout(sm, p.status);
                     break;
                 }
                 tc_fence_after();
                 bool ok = true;
                 for (int kt = 0; kt < p.kt_total; ++kt) {
-                    if (!mbar_wait_bounded(smem_u32(&sm->full[stage]), phase, WAIT_LIMIT_NS) ||
-                        !mbar_wait_bounded(smem_u32(&sm->sf_ready[stage]), phase, WAIT_LIMIT_NS)) {
+                    if (!mbar_wait_bounded(smem_u32(&sm->full[stage]), phase, p.wait_limit_ns) ||
+                        !mbar_wait_bounded(smem_u32(&sm->sf_ready[stage]), phase, p.wait_limit_ns)) {
                         raise_timeout(sm, p.status);
                         ok = false;
                         break;
@@ -318,7 +322,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             }
             // let every tcgen05 operation this thread issued finish before TMEM is freed
             tc_commit(smem_u32(&sm->drain));
-            if (!mbar_wait_bounded(smem_u32(&sm->drain), 0, WAIT_LIMIT_NS))
+            if (!mbar_wait_bounded(smem_u32(&sm->drain), 0, p.wait_limit_ns))
                 raise_timeout(sm, p.status);
         }
     } else if (warp == 2) {
@@ -331,7 +335,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 for (int kt = 0; kt < p.kt_total; ++kt) {
                     // The stage's TMEM scale buffer is free: the producer only refilled this
                     // stage after the MMAs that read the buffer last time had completed.
-                    if (!mbar_wait_bounded(smem_u32(&sm->full[stage]), phase, WAIT_LIMIT_NS)) {
+                    if (!mbar_wait_bounded(smem_u32(&sm->full[stage]), phase, p.wait_limit_ns)) {
                         raise_timeout(sm, p.status);
                         ok = false;
                         break;
@@ -371,7 +375,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             int m_blk, n_blk;
             tile_coords(p, tile, m_blk, n_blk);
             const int m0 = m_blk * BM, n0 = n_blk * BN;
-            const bool ok = mbar_wait_bounded(smem_u32(&sm->acc_full), local & 1, WAIT_LIMIT_NS);
+            const bool ok = mbar_wait_bounded(smem_u32(&sm->acc_full), local & 1, p.wait_limit_ns);
             if (!__all_sync(0xFFFFFFFFu, ok)) {
                 if (lane == 0)
                     raise_timeout(sm, p.status);
@@ -441,7 +445,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 alpha[lane + 32 * j] = column_alpha(p, ga, n0 + hc * HALF_N + lane + 32 * j);
             __syncwarp();
             // every lane waits (bounded); the vote keeps the warp's decision uniform
-            const bool ok = mbar_wait_bounded(smem_u32(&sm->acc_full), local & 1, WAIT_LIMIT_NS);
+            const bool ok = mbar_wait_bounded(smem_u32(&sm->acc_full), local & 1, p.wait_limit_ns);
             if (!__all_sync(0xFFFFFFFFu, ok)) {
                 if (lane == 0)
                     raise_timeout(sm, p.status);

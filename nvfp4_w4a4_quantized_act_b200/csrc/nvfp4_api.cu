@@ -237,6 +237,8 @@ int run_gemm(DeviceState *d, const uint8_t *a_codes, const uint8_t *a_sf, const 
     p.status = d->status;
     // re-stream the smaller operand: A is M x K/2 bytes of codes, W is N x K/2
     p.n_fastest = (M > N) ? 1 : 0;
+    p.inject_stall = (flags & NVFP4_DEBUG_INJECT_STALL) ? 1 : 0;
+    p.wait_limit_ns = p.inject_stall ? 20000000ull : WAIT_LIMIT_NS;
     const int grid = static_cast<int>(std::min<int64_t>(p.num_tiles, d->sm_count));
     if (h_amax != nullptr) {
         p.F = static_cast<int32_t>(N / 2);
@@ -367,7 +369,7 @@ int nvfp4_gemm_prequant(const uint8_t *a_codes, const uint8_t *a_sf, const float
                         const uint8_t *w_codes, const uint8_t *w_sf, int64_t N, const nvfp4_segment *segs,
                         const float *g_w, int nseg, void *out, unsigned flags, void *stream)
 {
-    if ((flags & ~(NVFP4_STATIC_SCALE | NVFP4_OUT_FP32)) != 0)
+    if ((flags & ~(NVFP4_STATIC_SCALE | NVFP4_OUT_FP32 | NVFP4_DEBUG_INJECT_STALL)) != 0)
         return NVFP4_ERR_INVALID_ARG;
     int rc = check_gemm_shape(M, N, K);
     if (rc != NVFP4_OK)

@@ -19,6 +19,7 @@ LIB_PATH = os.path.join(_PKG, "libnvfp4.so")
 NVFP4_STATIC_SCALE = 1
 NVFP4_OUT_FP32 = 2
 NVFP4_AMAX_GIVEN = 4
+NVFP4_DEBUG_INJECT_STALL = 1 << 30
 MAX_SEGMENTS = 16
 
 STATUS_NAMES = {
@@ -205,14 +206,15 @@ def quantize_act(X: torch.Tensor, g_a: torch.Tensor | None = None, static_scale:
     return codes[: M * K // 2].view(M, K // 2), sf, g_a
 
 
-def gemm_prequant(a_codes, a_sf, g_a, M: int, K: int, w: QuantizedWeight, out=None, out_fp32=False, stream=None):
+def gemm_prequant(a_codes, a_sf, g_a, M: int, K: int, w: QuantizedWeight, out=None, out_fp32=False, stream=None,
+                  debug_flags: int = 0):
     """nvfp4_gemm_prequant on already-quantized activations."""
     _require_cuda(a_codes, a_sf, g_a)
     dt = torch.float32 if out_fp32 else torch.bfloat16
     if out is None:
         out = torch.empty((M, w.N), dtype=dt, device=a_codes.device)
     arr, n = _segs(w.segments)
-    flags = NVFP4_OUT_FP32 if out_fp32 else 0
+    flags = (NVFP4_OUT_FP32 if out_fp32 else 0) | debug_flags
     _check(lib().nvfp4_gemm_prequant(_p(a_codes), _p(a_sf), _p(g_a), M, K, _p(w.codes), _p(w.sf), w.N, arr,
                                      _p(w.g_w), n, _p(out), flags, _stream(stream)), "nvfp4_gemm_prequant")
     return out

@@ -1,0 +1,51 @@
+"""bench.py's replica mode on CPU with world size 2 over gloo: every rank
+joins the barrier, the step time is the maximum over ranks and the reported
+throughput counts the work of all ranks (weak scaling)."""
+import os
+import socket
+import sys
+
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world),
+                      LOCAL_RANK=str(rank))
+    sys.path.insert(0, ROOT)
+    import bench
+    import torch.distributed as dist
+    r, w, _ = bench.dist_setup(None)
+    bench.barrier(w)
+    elapsed = bench.max_over_ranks(10.0 * (r + 1), w)  # rank 1 is the slower one
+    value = bench.aggregate_throughput(1.0e12, w, elapsed)
+    q.put((r, w, elapsed, value))
+    dist.destroy_process_group()
+
+
+@pytest.mark.timeout(120)
+def test_replicas_take_max_time_and_sum_work():
+    world = 2
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=90) for _ in range(world))
+    for p in procs:
+        p.join(timeout=30)
+        assert p.exitcode == 0
+    for r, w, elapsed, value in res:
+        assert w == world
+        assert elapsed == 20.0
+        # 2 ranks x 1 TFLOP in 20 ms per step -> 100 TFLOPS
+        assert abs(value - 100.0) < 1e-9
