@@ -13,8 +13,11 @@
 // (same page, "The abstract" and "The deep dive").
 //
 // Tile 128 x 256 (x 256 of K per pipeline stage), one CTA per SM, 12 warps:
-//   warp 0      TMA producer: codes by 2-D tiled TMA (128-byte swizzle),
-//               scale-factor tiles by 1-D bulk copies, 4-stage ring.
+//   warps 0, 3  TMA producers (4-stage ring): warp 0 the activation codes
+//               (2-D tiled TMA, 128-byte swizzle) and their scale tiles (1-D
+//               bulk copies), warp 3 the weight codes and scale tiles.  One
+//               issuing thread cannot stream a stage's 54 KB as fast as the
+//               MMAs consume it; two independent issuers can.
 //   warp 1      allocates 512 TMEM columns; one lane issues the MMAs.  The
 //               256-column tile is two 128-column accumulators and the
 //               128x128x64 kind::mxf4nvf4 MMAs alternate between them:
@@ -216,7 +219,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
-            mbar_init(smem_u32(&sm->full[s]), 1);
+            mbar_init(smem_u32(&sm->full[s]), 2);  // one arrival per producer warp
             mbar_init(smem_u32(&sm->empty[s]), 1);
             mbar_init(smem_u32(&sm->sf_ready[s]), 1);
         }
@@ -226,9 +229,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         sm->abort_flag = 0;
         fence_mbarrier_init();
     }
-    if (warp == 0 && lane == 0) {
-        prefetch_tensormap(&tmA);
-        prefetch_tensormap(&tmB);
+    if ((warp == 0 || warp == 3) && lane == 0) {
+        prefetch_tensormap(warp == 0 ? &tmA : &tmB);
     }
     if (warp == 1) {
         tmem_alloc(smem_u32(&sm->tmem_base), TMEM_COLS);
@@ -239,8 +241,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     tc_fence_after();
     const uint32_t tmem = sm->tmem_base;
 
-    if (warp == 0) {
-        // ------------------------------------------------------ producer
+    if (warp == 0 || warp == 3) {
+        // ----------------------------------------------------- producers
+        // Two warps share the loads of a stage: warp 0 the activation tile and
+        // its scales, warp 3 the weight tile and its scales.  One thread's
+        // stream of TMA instructions is slower than the stage's bytes need;
+        // two independent issuers double it.  Each arrives once on the
+        // stage's full barrier with its own byte count.
+        const bool w_side = (warp == 3);
         if (lane == 0 && !p.inject_stall) {
             int stage = 0;
             uint32_t phase = 0;
@@ -258,16 +266,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     const int nkb = min(KB_PER_STAGE, p.kb_total - kt * KB_PER_STAGE);
                     const uint32_t sf_bytes = nkb * SF_TILE;
                     const uint32_t bar = smem_u32(&sm->full[stage]);
-                    mbar_arrive_expect_tx(bar, A_BYTES + B_BYTES + sf_bytes * (1 + nb_tiles));
-                    tma_load_2d(a_smem(stage), &tmA, kt * BK_BYTES, m0, bar);
-                    tma_load_2d(b_smem(stage), &tmB, kt * BK_BYTES, n0, bar);
-                    bulk_load(sfa_smem(stage),
-                              p.sfa + (static_cast<int64_t>(m_blk) * p.kb_total + kt * KB_PER_STAGE) * SF_TILE,
-                              sf_bytes, bar);
-                    for (int j = 0; j < nb_tiles; ++j)
-                        bulk_load(sfb_smem(stage) + j * (KB_PER_STAGE * SF_TILE),
-                                  p.sfb + (static_cast<int64_t>(rb0 + j) * p.kb_total + kt * KB_PER_STAGE) * SF_TILE,
+                    if (!w_side) {
+                        mbar_arrive_expect_tx(bar, A_BYTES + sf_bytes);
+                        tma_load_2d(a_smem(stage), &tmA, kt * BK_BYTES, m0, bar);
+                        bulk_load(sfa_smem(stage),
+                                  p.sfa + (static_cast<int64_t>(m_blk) * p.kb_total + kt * KB_PER_STAGE) * SF_TILE,
                                   sf_bytes, bar);
+                    } else {
+                        mbar_arrive_expect_tx(bar, B_BYTES + sf_bytes * nb_tiles);
+                        tma_load_2d(b_smem(stage), &tmB, kt * BK_BYTES, n0, bar);
+                        for (int j = 0; j < nb_tiles; ++j)
+                            bulk_load(sfb_smem(stage) + j * (KB_PER_STAGE * SF_TILE),
+                                      p.sfb + (static_cast<int64_t>(rb0 + j) * p.kb_total + kt * KB_PER_STAGE) * SF_TILE,
+                                      sf_bytes, bar);
+                    }
                     if (++stage == STAGES) {
                         stage = 0;
                         phase ^= 1u;
