@@ -77,6 +77,8 @@ struct Params {
     int32_t kb_total;    // K / 64
     int32_t kt_total;    // ceil(kb_total / 4)
     int32_t n_row_tiles; // ceil(N / 128): scale tiles of W per K-step
+    uint32_t sf_box_bytes;  // bytes of one scale row-tile per stage (2 KB unless K < 256)
+    uint32_t sfb_box_rows;  // scale row-tiles of W per stage load (2, or 1 when N <= 128)
     const uint8_t *sfa;
     const uint8_t *sfb;
     const float *g_a;
@@ -203,6 +205,7 @@ __device__ __forceinline__ float silu_mul(float g, float u)
 template <bool GATED>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                     const __grid_constant__ CUtensorMap tmSFA, const __grid_constant__ CUtensorMap tmSFB,
                      const __grid_constant__ Params p)
 {
     extern __shared__ uint8_t smem_raw[];
@@ -231,6 +234,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     if ((warp == 0 || warp == 3) && lane == 0) {
         prefetch_tensormap(warp == 0 ? &tmA : &tmB);
+        prefetch_tensormap(warp == 0 ? &tmSFA : &tmSFB);
     }
     if (warp == 1) {
         tmem_alloc(smem_u32(&sm->tmem_base), TMEM_COLS);
@@ -257,28 +261,26 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 tile_coords(p, tile, m_blk, n_blk);
                 const int m0 = m_blk * BM, n0 = n_blk * BN;
                 const int rb0 = n0 >> 7;  // first 128-row scale tile of W
-                const int nb_tiles = (rb0 + 1 < p.n_row_tiles) ? 2 : 1;
                 for (int kt = 0; kt < p.kt_total; ++kt) {
                     if (!mbar_wait_bounded(smem_u32(&sm->empty[stage]), phase ^ 1u, p.wait_limit_ns)) {
                         raise_timeout(sm, p.status);
                         break;
                     }
-                    const int nkb = min(KB_PER_STAGE, p.kb_total - kt * KB_PER_STAGE);
-                    const uint32_t sf_bytes = nkb * SF_TILE;
+                    // Scale tiles come as 2-D boxes of 8-byte elements over the
+                    // [row tile][K/64 x 512 B] scale array: one instruction for
+                    // the stage's 4 K-steps (both W row tiles at once).  A box
+                    // reaching past the last K-step or row tile is zero-filled and
+                    // still counts its full size.
                     const uint32_t bar = smem_u32(&sm->full[stage]);
+                    const int32_t sf_x = kt * KB_PER_STAGE * (SF_TILE / 8);
                     if (!w_side) {
-                        mbar_arrive_expect_tx(bar, A_BYTES + sf_bytes);
+                        mbar_arrive_expect_tx(bar, A_BYTES + p.sf_box_bytes);
                         tma_load_2d(a_smem(stage), &tmA, kt * BK_BYTES, m0, bar);
-                        bulk_load(sfa_smem(stage),
-                                  p.sfa + (static_cast<int64_t>(m_blk) * p.kb_total + kt * KB_PER_STAGE) * SF_TILE,
-                                  sf_bytes, bar);
+                        tma_load_2d(sfa_smem(stage), &tmSFA, sf_x, m_blk, bar);
                     } else {
-                        mbar_arrive_expect_tx(bar, B_BYTES + sf_bytes * nb_tiles);
+                        mbar_arrive_expect_tx(bar, B_BYTES + p.sf_box_bytes * p.sfb_box_rows);
                         tma_load_2d(b_smem(stage), &tmB, kt * BK_BYTES, n0, bar);
-                        for (int j = 0; j < nb_tiles; ++j)
-                            bulk_load(sfb_smem(stage) + j * (KB_PER_STAGE * SF_TILE),
-                                      p.sfb + (static_cast<int64_t>(rb0 + j) * p.kb_total + kt * KB_PER_STAGE) * SF_TILE,
-                                      sf_bytes, bar);
+                        tma_load_2d(sfb_smem(stage), &tmSFB, sf_x, rb0, bar);
                     }
                     if (++stage == STAGES) {
                         stage = 0;
@@ -360,7 +362,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                         tc_cp_32x128b_x4(sfa_t + kb * 4, smem_desc(sfa_smem(stage) + kb * SF_TILE, 0, 128, 0));
                         tc_cp_32x128b_x4(sfb_t + kb * 8, smem_desc(sfb_smem(stage) + kb * SF_TILE, 0, 128, 0));
                         tc_cp_32x128b_x4(sfb_t + kb * 8 + 4,
-                                         smem_desc(sfb_smem(stage) + (KB_PER_STAGE + kb) * SF_TILE, 0, 128, 0));
+                                         smem_desc(sfb_smem(stage) + p.sf_box_bytes + kb * SF_TILE, 0, 128, 0));
                     }
                     tc_commit(smem_u32(&sm->sf_ready[stage]));
                     if (++stage == STAGES) {

@@ -200,6 +200,25 @@ int make_codes_map(CUtensorMap *map, const uint8_t *codes, int64_t rows, int64_t
     return r == CUDA_SUCCESS ? NVFP4_OK : NVFP4_ERR_CUDA;
 }
 
+// Scale factors of a [rows, K] operand as a 2-D array of 8-byte elements:
+// row = one 128-row tile, K/64 * 512 bytes long.  A box is one stage's
+// 4 K-steps (2 KB; the whole row when K < 256) of box_rows row tiles.
+int make_sf_map(CUtensorMap *map, const uint8_t *sf, int64_t row_tiles, int64_t kb_total, uint32_t box_rows,
+                uint32_t *box_bytes)
+{
+    const int64_t inner = kb_total * 64;
+    const uint32_t box_inner = static_cast<uint32_t>(std::min<int64_t>(inner, 256));
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(row_tiles)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(kb_total * 512)};
+    cuuint32_t box[2] = {box_inner, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT64, 2, const_cast<uint8_t *>(sf), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    *box_bytes = box_inner * 8;
+    return r == CUDA_SUCCESS ? NVFP4_OK : NVFP4_ERR_CUDA;
+}
+
 // h_amax != nullptr selects the gated MLP epilogue (W is [gate | up]
 // interleaved in 128-row blocks, N = 2F, out = h [M, F] bf16).
 int run_gemm(DeviceState *d, const uint8_t *a_codes, const uint8_t *a_sf, const float *g_a, int64_t M, int64_t K,
@@ -209,8 +228,17 @@ int run_gemm(DeviceState *d, const uint8_t *a_codes, const uint8_t *a_sf, const 
     using namespace nvfp4::gemm;
     if (M == 0 || N == 0)
         return NVFP4_OK;
-    CUtensorMap tmA, tmB;
-    if (make_codes_map(&tmA, a_codes, M, K, BM) != NVFP4_OK || make_codes_map(&tmB, w_codes, N, K, BN) != NVFP4_OK)
+    // every operand is read by TMA, which needs 16-byte aligned bases (the
+    // entry points check this already; internal callers pass workspace slices)
+    if (!aligned16(a_codes) || !aligned16(w_codes) || !aligned16(a_sf) || !aligned16(w_sf))
+        return NVFP4_ERR_MISALIGNED;
+    const int64_t n_row_tiles = cdiv(N, 128);
+    const uint32_t sfb_rows = n_row_tiles >= 2 ? 2u : 1u;
+    CUtensorMap tmA, tmB, tmSFA, tmSFB;
+    uint32_t sf_box = 0, sf_box_b = 0;
+    if (make_codes_map(&tmA, a_codes, M, K, BM) != NVFP4_OK || make_codes_map(&tmB, w_codes, N, K, BN) != NVFP4_OK ||
+        make_sf_map(&tmSFA, a_sf, cdiv(M, 128), K / 64, 1, &sf_box) != NVFP4_OK ||
+        make_sf_map(&tmSFB, w_sf, n_row_tiles, K / 64, sfb_rows, &sf_box_b) != NVFP4_OK)
         return NVFP4_ERR_CUDA;
     Params p;
     std::memset(&p, 0, sizeof(p));
@@ -222,7 +250,9 @@ int run_gemm(DeviceState *d, const uint8_t *a_codes, const uint8_t *a_sf, const 
     p.num_tiles = p.num_m * p.num_n;
     p.kb_total = static_cast<int32_t>(K / 64);
     p.kt_total = static_cast<int32_t>(cdiv(K / 64, KB_PER_STAGE));
-    p.n_row_tiles = static_cast<int32_t>(cdiv(N, 128));
+    p.n_row_tiles = static_cast<int32_t>(n_row_tiles);
+    p.sf_box_bytes = sf_box;
+    p.sfb_box_rows = sfb_rows;
     p.sfa = a_sf;
     p.sfb = w_sf;
     p.g_a = g_a;
@@ -244,9 +274,9 @@ int run_gemm(DeviceState *d, const uint8_t *a_codes, const uint8_t *a_sf, const 
         p.F = static_cast<int32_t>(N / 2);
         p.h_amax = h_amax;
         p.vec_ok = aligned16(out) && ((p.F * 2) % 16 == 0);
-        gemm_nvf4_kernel<true><<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(tmA, tmB, p);
+        gemm_nvf4_kernel<true><<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(tmA, tmB, tmSFA, tmSFB, p);
     } else {
-        gemm_nvf4_kernel<false><<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(tmA, tmB, p);
+        gemm_nvf4_kernel<false><<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(tmA, tmB, tmSFA, tmSFB, p);
     }
     g_launches++;
     return launch_ok();
