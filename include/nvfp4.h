@@ -87,6 +87,10 @@ typedef struct {
                                * skipped so its bounded waits run out (20 ms) and it
                                * unwinds, latching NVFP4_ERR_TIMEOUT; outputs are not
                                * written.  Exercises the failure path without a hang. */
+#define NVFP4_SINGLE_CTA (1u << 29) /* GEMM entry points: use the one-CTA-per-tile kernel even
+                               * where the CTA-pair kernel would run (M > 128).  Both
+                               * compute the same block-scaled products; for tests and
+                               * comparisons. */
 #define NVFP4_AMAX_GIVEN 4u   /* nvfp4_quantize_act: the first word of ws already holds max|X|
                                * (bf16 magnitude bits, as nvfp4_gemm_prequant_swiglu leaves
                                * it); skip the amax pass */

@@ -33,6 +33,7 @@
 // when a wait runs out the kernel latches kStatusTimeout and unwinds.
 #pragma once
 
+#include <cstddef>
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -74,6 +75,7 @@ constexpr uint32_t IDESC = (1u << 7) | (1u << 10) | (uint32_t(HALF_N >> 3) << 17
 struct Params {
     int32_t M, N, K;
     int32_t num_m, num_n, num_tiles;
+    int32_t pair_m, pair_n, pair_tiles;  // 256 x 256 tiles of the CTA-pair kernel
     int32_t kb_total;    // K / 64
     int32_t kt_total;    // ceil(kb_total / 4)
     int32_t n_row_tiles; // ceil(N / 128): scale tiles of W per K-step
@@ -88,6 +90,7 @@ struct Params {
     void *out;
     int32_t out_fp32;
     int32_t vec_ok;      // rows of `out` are 16-byte aligned
+    int32_t tma_out;     // bf16 output stored by TMA from swizzled staging boxes (pair kernel)
     uint32_t *status;
     // gated MLP epilogue (template flag GATED): the weight is [gate F | up F]
     // interleaved in 128-row blocks; out is h [M, F] bf16 and the largest
@@ -125,13 +128,25 @@ struct Smem {
     uint64_t drain;
     uint32_t tmem_base;
     volatile int32_t abort_flag;
-    float alpha[EPI_THREADS / 32][HALF_N];  // per epilogue warp: alpha of its 128 columns
+    alignas(16) float alpha[EPI_THREADS / 32][HALF_N];  // per epilogue warp, read as float4
 };
+
+static_assert(offsetof(Smem, alpha) % 16 == 0, "alpha is read as float4");
 
 __device__ __forceinline__ void raise_timeout(Smem *sm, uint32_t *status)
 {
     sm->abort_flag = 1;
     atomicOr(status, kStatusTimeout);
+}
+
+// Module segment of output column n (n < N).
+__device__ __forceinline__ int column_segment(const Params &p, int32_t n)
+{
+    int s = 0;
+#pragma unroll 1
+    while (s + 1 < p.nseg && n >= p.seg_end[s])
+        ++s;
+    return s;
 }
 
 __device__ __forceinline__ float column_alpha(const Params &p, float ga, int32_t n)
@@ -193,6 +208,23 @@ __device__ __forceinline__ void store_64(const Params &p, const float *alpha, in
             for (int j = 0; j < 64 && col0 + j < p.N; ++j)
                 o[j] = __float2bfloat16_rn(__fmul_rn(__uint_as_float(v[j]), alpha[j]));
         }
+    }
+}
+
+// Store 128 bf16 values of one row (as 64 packed pairs) at [row, col0).
+__device__ __forceinline__ void store_bf16_packed_128(const Params &p, int32_t row, int32_t col0,
+                                                      const uint32_t (&pk)[64])
+{
+    if (row >= p.M || col0 >= p.N)
+        return;
+    __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(p.out) + static_cast<int64_t>(row) * p.N + col0;
+    if (p.vec_ok && col0 + 128 <= p.N) {
+#pragma unroll
+        for (int j = 0; j < 64; j += 4)
+            *reinterpret_cast<uint4 *>(o + 2 * j) = make_uint4(pk[j], pk[j + 1], pk[j + 2], pk[j + 3]);
+    } else {
+        for (int j = 0; j < 128 && col0 + j < p.N; ++j)
+            o[j] = __ushort_as_bfloat16(static_cast<unsigned short>((j & 1) ? (pk[j >> 1] >> 16) : (pk[j >> 1] & 0xFFFFu)));
     }
 }
 

@@ -12,6 +12,7 @@
 
 #include "nvfp4.h"
 #include "gemm_kernel.cuh"
+#include "gemm_pair_kernel.cuh"
 #include "quantize_kernels.cuh"
 
 namespace {
@@ -66,7 +67,11 @@ DeviceState *device_state()
         if (cudaFuncSetAttribute(nvfp4::gemm::gemm_nvf4_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  nvfp4::gemm::SMEM_BYTES) != cudaSuccess ||
             cudaFuncSetAttribute(nvfp4::gemm::gemm_nvf4_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 nvfp4::gemm::SMEM_BYTES) != cudaSuccess)
+                                 nvfp4::gemm::SMEM_BYTES) != cudaSuccess ||
+            cudaFuncSetAttribute(nvfp4::gemm::pair::gemm_nvf4_pair_kernel<false>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, nvfp4::gemm::pair::SMEM_BYTES) != cudaSuccess ||
+            cudaFuncSetAttribute(nvfp4::gemm::pair::gemm_nvf4_pair_kernel<true>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, nvfp4::gemm::pair::SMEM_BYTES) != cudaSuccess)
             return nullptr;
         d.gemm_attr_set = true;
         if (g_encode == nullptr) {
@@ -219,6 +224,20 @@ int make_sf_map(CUtensorMap *map, const uint8_t *sf, int64_t row_tiles, int64_t 
     return r == CUDA_SUCCESS ? NVFP4_OK : NVFP4_ERR_CUDA;
 }
 
+// bf16 output [rows, cols] as the TMA store target of the pair kernel's
+// epilogue: 32-row x 64-column boxes, 128-byte swizzle.
+int make_out_map(CUtensorMap *map, void *out, int64_t rows, int64_t cols)
+{
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols * 2)};
+    cuuint32_t box[2] = {64, 32};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, out, dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? NVFP4_OK : NVFP4_ERR_CUDA;
+}
+
 // h_amax != nullptr selects the gated MLP epilogue (W is [gate | up]
 // interleaved in 128-row blocks, N = 2F, out = h [M, F] bf16).
 int run_gemm(DeviceState *d, const uint8_t *a_codes, const uint8_t *a_sf, const float *g_a, int64_t M, int64_t K,
@@ -236,7 +255,10 @@ int run_gemm(DeviceState *d, const uint8_t *a_codes, const uint8_t *a_sf, const 
     const uint32_t sfb_rows = n_row_tiles >= 2 ? 2u : 1u;
     CUtensorMap tmA, tmB, tmSFA, tmSFB;
     uint32_t sf_box = 0, sf_box_b = 0;
-    if (make_codes_map(&tmA, a_codes, M, K, BM) != NVFP4_OK || make_codes_map(&tmB, w_codes, N, K, BN) != NVFP4_OK ||
+    // CTA pairs (256-row tiles) once A has more than one 128-row block
+    const bool use_pair = (M > BM) && !(flags & NVFP4_SINGLE_CTA);
+    if (make_codes_map(&tmA, a_codes, M, K, BM) != NVFP4_OK ||
+        make_codes_map(&tmB, w_codes, N, K, use_pair ? 128u : static_cast<uint32_t>(BN)) != NVFP4_OK ||
         make_sf_map(&tmSFA, a_sf, cdiv(M, 128), K / 64, 1, &sf_box) != NVFP4_OK ||
         make_sf_map(&tmSFB, w_sf, n_row_tiles, K / 64, sfb_rows, &sf_box_b) != NVFP4_OK)
         return NVFP4_ERR_CUDA;
@@ -248,6 +270,9 @@ int run_gemm(DeviceState *d, const uint8_t *a_codes, const uint8_t *a_sf, const 
     p.num_m = static_cast<int32_t>(cdiv(M, BM));
     p.num_n = static_cast<int32_t>(cdiv(N, BN));
     p.num_tiles = p.num_m * p.num_n;
+    p.pair_m = static_cast<int32_t>(cdiv(M, pair::PAIR_M));
+    p.pair_n = static_cast<int32_t>(cdiv(N, pair::PAIR_N));
+    p.pair_tiles = p.pair_m * p.pair_n;
     p.kb_total = static_cast<int32_t>(K / 64);
     p.kt_total = static_cast<int32_t>(cdiv(K / 64, KB_PER_STAGE));
     p.n_row_tiles = static_cast<int32_t>(n_row_tiles);
@@ -269,14 +294,35 @@ int run_gemm(DeviceState *d, const uint8_t *a_codes, const uint8_t *a_sf, const 
     p.n_fastest = (M > N) ? 1 : 0;
     p.inject_stall = (flags & NVFP4_DEBUG_INJECT_STALL) ? 1 : 0;
     p.wait_limit_ns = p.inject_stall ? 20000000ull : WAIT_LIMIT_NS;
-    const int grid = static_cast<int>(std::min<int64_t>(p.num_tiles, d->sm_count));
     if (h_amax != nullptr) {
         p.F = static_cast<int32_t>(N / 2);
         p.h_amax = h_amax;
         p.vec_ok = aligned16(out) && ((p.F * 2) % 16 == 0);
-        gemm_nvf4_kernel<true><<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(tmA, tmB, tmSFA, tmSFB, p);
+    }
+    if (use_pair) {
+        // bf16 outputs with 16-byte rows leave through TMA stores
+        CUtensorMap tmOut;
+        std::memset(&tmOut, 0, sizeof(tmOut));
+        p.tma_out = 0;
+        if (!p.out_fp32 && p.vec_ok) {
+            if (make_out_map(&tmOut, out, M, h_amax != nullptr ? N / 2 : N) != NVFP4_OK)
+                return NVFP4_ERR_CUDA;
+            p.tma_out = 1;
+        }
+        // one cluster of two CTAs per pair of SMs, persistent over the pair tiles
+        const int grid = 2 * static_cast<int>(std::min<int64_t>(p.pair_tiles, d->sm_count / 2));
+        if (h_amax != nullptr)
+            pair::gemm_nvf4_pair_kernel<true><<<grid, pair::NUM_THREADS, pair::SMEM_BYTES, stream>>>(
+                tmA, tmB, tmSFA, tmSFB, tmOut, p);
+        else
+            pair::gemm_nvf4_pair_kernel<false><<<grid, pair::NUM_THREADS, pair::SMEM_BYTES, stream>>>(
+                tmA, tmB, tmSFA, tmSFB, tmOut, p);
     } else {
-        gemm_nvf4_kernel<false><<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(tmA, tmB, tmSFA, tmSFB, p);
+        const int grid = static_cast<int>(std::min<int64_t>(p.num_tiles, d->sm_count));
+        if (h_amax != nullptr)
+            gemm_nvf4_kernel<true><<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(tmA, tmB, tmSFA, tmSFB, p);
+        else
+            gemm_nvf4_kernel<false><<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(tmA, tmB, tmSFA, tmSFB, p);
     }
     g_launches++;
     return launch_ok();
@@ -399,7 +445,7 @@ int nvfp4_gemm_prequant(const uint8_t *a_codes, const uint8_t *a_sf, const float
                         const uint8_t *w_codes, const uint8_t *w_sf, int64_t N, const nvfp4_segment *segs,
                         const float *g_w, int nseg, void *out, unsigned flags, void *stream)
 {
-    if ((flags & ~(NVFP4_STATIC_SCALE | NVFP4_OUT_FP32 | NVFP4_DEBUG_INJECT_STALL)) != 0)
+    if ((flags & ~(NVFP4_STATIC_SCALE | NVFP4_OUT_FP32 | NVFP4_DEBUG_INJECT_STALL | NVFP4_SINGLE_CTA)) != 0)
         return NVFP4_ERR_INVALID_ARG;
     int rc = check_gemm_shape(M, N, K);
     if (rc != NVFP4_OK)
@@ -436,7 +482,7 @@ int nvfp4_linear_fused(const void *X, int64_t M, int64_t K, const uint8_t *w_cod
                        const nvfp4_segment *segs, const float *g_w, int nseg, void *out, unsigned flags, void *ws,
                        size_t ws_bytes, void *stream)
 {
-    if ((flags & ~(NVFP4_STATIC_SCALE | NVFP4_OUT_FP32)) != 0)
+    if ((flags & ~(NVFP4_STATIC_SCALE | NVFP4_OUT_FP32 | NVFP4_SINGLE_CTA)) != 0)
         return NVFP4_ERR_INVALID_ARG;
     int rc = check_gemm_shape(M, N, K);
     if (rc != NVFP4_OK)
@@ -752,7 +798,7 @@ extern "C" int nvfp4_linear_swiglu(const void *X, int64_t M, int64_t K, const ui
                                    int64_t F, const float *g_w, void *h, uint8_t *h_codes, uint8_t *h_sf, float *g_h,
                                    unsigned flags, void *ws, size_t ws_bytes, void *stream)
 {
-    if ((flags & ~static_cast<unsigned>(NVFP4_STATIC_SCALE)) != 0)
+    if ((flags & ~(NVFP4_STATIC_SCALE | NVFP4_SINGLE_CTA)) != 0)
         return NVFP4_ERR_INVALID_ARG;
     int rc = check_gemm_shape(M, 2 * F, K);
     if (rc != NVFP4_OK)
@@ -796,7 +842,7 @@ extern "C" int nvfp4_linear_swiglu(const void *X, int64_t M, int64_t K, const ui
     nvfp4::SegRows gu;
     const nvfp4_segment two[2] = {{0, F}, {F, 2 * F}};
     check_segments(two, 2, 2 * F, &gu);
-    rc = run_gemm(d, a_codes, a_sf, g_a, M, K, w_codes, w_sf, 2 * F, gu, g_w, h, 0, s, h_amax);
+    rc = run_gemm(d, a_codes, a_sf, g_a, M, K, w_codes, w_sf, 2 * F, gu, g_w, h, flags & NVFP4_SINGLE_CTA, s, h_amax);
     if (rc != NVFP4_OK)
         return rc;
     // h -> NVFP4 with the dynamic scale folded in by the epilogue

@@ -20,6 +20,7 @@ NVFP4_STATIC_SCALE = 1
 NVFP4_OUT_FP32 = 2
 NVFP4_AMAX_GIVEN = 4
 NVFP4_DEBUG_INJECT_STALL = 1 << 30
+NVFP4_SINGLE_CTA = 1 << 29
 MAX_SEGMENTS = 16
 
 STATUS_NAMES = {
@@ -221,7 +222,7 @@ def gemm_prequant(a_codes, a_sf, g_a, M: int, K: int, w: QuantizedWeight, out=No
 
 
 def linear_fused(X: torch.Tensor, w: QuantizedWeight, out=None, out_fp32=False, ws=None, static_scale=False,
-                 stream=None):
+                 stream=None, single_cta=False):
     """nvfp4_linear_fused: quantize X on the fly, fused-module GEMM with one
     global scale per module segment."""
     _require_cuda(X)
@@ -235,6 +236,7 @@ def linear_fused(X: torch.Tensor, w: QuantizedWeight, out=None, out_fp32=False, 
         ws = _empty_u8(workspace_bytes(M, w.N, K, len(w.segments)), X.device)
     arr, n = _segs(w.segments)
     flags = (NVFP4_OUT_FP32 if out_fp32 else 0) | (NVFP4_STATIC_SCALE if static_scale else 0)
+    flags |= NVFP4_SINGLE_CTA if single_cta else 0
     _check(lib().nvfp4_linear_fused(_p(X), M, K, _p(w.codes), _p(w.sf), w.N, arr, _p(w.g_w), n, _p(out), flags,
                                     _p(ws), ws.numel(), _stream(stream)), "nvfp4_linear_fused")
     return out
@@ -329,7 +331,7 @@ def quantize_weights_gated(W: torch.Tensor, stream=None) -> QuantizedWeight:
 
 
 def linear_swiglu(X: torch.Tensor, w: QuantizedWeight, h=None, h_codes=None, h_sf=None, g_h=None, ws=None,
-                  static_scale=False, stream=None):
+                  static_scale=False, stream=None, single_cta=False):
     """nvfp4_linear_swiglu -> (h bf16 [M, F], h_codes [M, F/2], h_sf, g_h)."""
     _require_cuda(X)
     assert w.gated and X.dtype == torch.bfloat16 and X.is_contiguous()
@@ -346,7 +348,7 @@ def linear_swiglu(X: torch.Tensor, w: QuantizedWeight, h=None, h_codes=None, h_s
         g_h = torch.empty(1, dtype=torch.float32, device=dev)
     if ws is None:
         ws = _empty_u8(workspace_bytes(M, w.N, K, 2), dev)
-    flags = NVFP4_STATIC_SCALE if static_scale else 0
+    flags = (NVFP4_STATIC_SCALE if static_scale else 0) | (NVFP4_SINGLE_CTA if single_cta else 0)
     _check(lib().nvfp4_linear_swiglu(_p(X), M, K, _p(w.codes), _p(w.sf), F, _p(w.g_w), _p(h), _p(h_codes),
                                      _p(h_sf), _p(g_h), flags, _p(ws), ws.numel(), _stream(stream)),
            "nvfp4_linear_swiglu")

@@ -1,7 +1,9 @@
 """Block-scaled FP4 GEMM on the tensor cores against the oracle's fp64 GEMM
 over the same (oracle-quantized) operands: every output within
 1e-5 * sum|a*b| + 1e-6; bf16 outputs equal the RNE rounding of the fp32
-path; exact-integer problems bit-exact."""
+path; exact-integer problems bit-exact.  Shapes with M > 128 run on the
+CTA-pair kernel by default; each check also runs the one-CTA kernel
+(NVFP4_SINGLE_CTA) on the same operands."""
 import numpy as np
 import pytest
 import torch
@@ -15,12 +17,15 @@ from nvfp4_testutil import (DEV, bf16_of_f32, check_gemm, dev_u8, host, oracle_a
 pytestmark = pytest.mark.gpu
 
 
-def _run(xb, wb, segments):
+KERNELS = {"auto": 0, "single_cta": ops.NVFP4_SINGLE_CTA}
+
+
+def _run(xb, wb, segments, flags=0):
     M, K = xb.shape
     (ac, asf, ga), (oc, os_, og) = oracle_act_on_device(xb)
     qw, (wc, ws, wg) = oracle_weight_on_device(wb, segments)
-    out32 = ops.gemm_prequant(ac, asf, ga, M, K, qw, out_fp32=True)
-    out16 = ops.gemm_prequant(ac, asf, ga, M, K, qw)
+    out32 = ops.gemm_prequant(ac, asf, ga, M, K, qw, out_fp32=True, debug_flags=flags)
+    out16 = ops.gemm_prequant(ac, asf, ga, M, K, qw, debug_flags=flags)
     torch.cuda.synchronize()
     grow = oracle.rows_scale(segments, wg, wb.shape[0])
     C, B = oracle.linear_full(oc, os_, og, wc, ws, grow)
@@ -40,11 +45,12 @@ SHAPES = [
 ]
 
 
+@pytest.mark.parametrize("kernel", sorted(KERNELS))
 @pytest.mark.parametrize("M,N,K", SHAPES)
-def test_ragged_shapes(M, N, K):
+def test_ragged_shapes(M, N, K, kernel):
     X = wl.activation_normal(M, K, seed=M + N + K, n_outliers=min(4, K // 16), scale=50.0)
     W = wl.weight_normal(N, K, 0.02, seed=3 * N + K)
-    o32, o16, C, B = _run(wl.bf16_bits(X), wl.bf16_bits(W), [(0, N)])
+    o32, o16, C, B = _run(wl.bf16_bits(X), wl.bf16_bits(W), [(0, N)], KERNELS[kernel])
     check_gemm(o32, C, B, f"{M}x{N}x{K}")
     assert np.array_equal(o16, bf16_of_f32(o32))
 
@@ -53,8 +59,9 @@ def _pack(cu):
     return (cu[:, 0::2] | (cu[:, 1::2] << 4)).astype(np.uint8)
 
 
-@pytest.mark.parametrize("M,N,K", [(128, 192, 256), (200, 400, 1024), (64, 130, 4096)])
-def test_exact_integer_problem_bit_exact(M, N, K):
+@pytest.mark.parametrize("kernel", sorted(KERNELS))
+@pytest.mark.parametrize("M,N,K", [(128, 192, 256), (200, 400, 1024), (64, 130, 4096), (520, 700, 1280)])
+def test_exact_integer_problem_bit_exact(M, N, K, kernel):
     """Codes in {0, +-1, +-2, +-4}, every scale 1.0, g = 1: all partial sums
     are integers below 2^24, so the tensor-core result must be exact."""
     rng = np.random.default_rng(M * N)
@@ -69,12 +76,13 @@ def test_exact_integer_problem_bit_exact(M, N, K):
                              torch.ones(1, dtype=torch.float32, device=DEV), [(0, N)], N, K)
     g1 = torch.ones(1, dtype=torch.float32, device=DEV)
     out = ops.gemm_prequant(dev_u8(a_codes).view(M, K // 2), dev_u8(oracle.swizzle(sa, K)), g1, M, K, qw,
-                            out_fp32=True)
+                            out_fp32=True, debug_flags=KERNELS[kernel])
     want = oracle.e2m1_table()[ca].astype(np.int64) @ oracle.e2m1_table()[cw].astype(np.int64).T
     assert np.array_equal(host(out).astype(np.float64), want.astype(np.float64))
 
 
-def test_scale_layout_drives_the_mma():
+@pytest.mark.parametrize("kernel", sorted(KERNELS))
+def test_scale_layout_drives_the_mma(kernel):
     """Distinct power-of-two scales per block and row: any mistake in the
     scale-factor layout or its TMEM placement changes the result."""
     rng = np.random.default_rng(21)
@@ -87,7 +95,7 @@ def test_scale_layout_drives_the_mma():
                              torch.ones(1, dtype=torch.float32, device=DEV), [(0, N)], N, K)
     g1 = torch.ones(1, dtype=torch.float32, device=DEV)
     out = ops.gemm_prequant(dev_u8(_pack(ca)).view(M, K // 2), dev_u8(oracle.swizzle(sa, K)), g1, M, K, qw,
-                            out_fp32=True)
+                            out_fp32=True, debug_flags=KERNELS[kernel])
     C, B = oracle.linear_full(_pack(ca), sa, 1.0, _pack(cw), sw, np.float32(1.0))
     assert np.array_equal(host(out).astype(np.float64), C)
 

@@ -44,9 +44,9 @@ def _h_tolerance(Cg, Bg, Cu, Bu, h_ref):
     return 1.1 * tg * (np.abs(Cu) + tu) + s * tu + 1e-6 * np.abs(h_ref) + 0.5 * ulp * (1 + 1e-6) + 1e-30
 
 
-def _check(M, K, F, X, W, rows, cols):
+def _check(M, K, F, X, W, rows, cols, single_cta=False):
     qw = ops.quantize_weights_gated(W.to(DEV))
-    h, hc, hsf, gh = ops.linear_swiglu(X.to(DEV), qw)
+    h, hc, hsf, gh = ops.linear_swiglu(X.to(DEV), qw, single_cta=single_cta)
     assert ops.get_status() == 0
     xb, wb = wl.bf16_bits(X), wl.bf16_bits(W)
     g_a = oracle.global_scale(oracle.amax(xb))
@@ -71,11 +71,13 @@ def _check(M, K, F, X, W, rows, cols):
     assert np.array_equal(oracle.unswizzle(host(hsf), M, F)[rows], s_ref)
 
 
-def test_linear_swiglu_small_full_check():
-    M, K, F = 200, 512, 384
-    X = wl.activation_normal(M, K, 51)
-    W = _gate_up(F, K, 52)
-    _check(M, K, F, X, W, np.arange(M), np.arange(F))
+@pytest.mark.parametrize("single_cta", [False, True])
+@pytest.mark.parametrize("M,K,F", [(200, 512, 384), (300, 768, 640)])
+def test_linear_swiglu_small_full_check(M, K, F, single_cta):
+    """Every h value: M > 128 runs the CTA-pair kernel unless single_cta."""
+    X = wl.activation_normal(M, K, 51 + M)
+    W = _gate_up(F, K, 52 + F)
+    _check(M, K, F, X, W, np.arange(M), np.arange(F), single_cta)
 
 
 def test_linear_swiglu_prefill_mlp_full_size():
