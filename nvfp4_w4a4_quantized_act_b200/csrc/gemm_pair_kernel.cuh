@@ -26,7 +26,7 @@
 //   warps 4..7  scale copiers (leader only): warp 4 + kb copies K-step kb's A
 //               tile and both W tiles into both CTAs' TMEM (pair-mode
 //               tcgen05.cp reads each CTA's own shared memory) and commits to
-//               sf_ready.  While MMAs occupy the tensor pipe a copy takes its
+//               the stage's full barrier.  While MMAs occupy the tensor pipe a copy takes its
 //               issuing thread about 70 cycles; twelve per stage from one
 //               thread (or from the MMA thread itself) would outlast the
 //               stage's MMAs, four threads overlap them.
@@ -69,6 +69,11 @@ constexpr int WRITER_WARP0 = 4;
 constexpr int EPI_WARP0 = 8;
 constexpr int EPI_WARPS = 8;
 constexpr uint32_t SF_READY_COUNT = KB_PER_STAGE;         // one commit per copier warp
+// full[stage]: the leader's A and W producers (arrive with the stage's byte
+// count) and the four copier warps (commit once their copies are done).  One
+// barrier per stage: a satisfied mbarrier wait still costs the MMA thread
+// ~70 cycles, and the pipe holds only about one MMA of queued work.
+constexpr uint32_t FULL_COUNT = 2 + SF_READY_COUNT;
 constexpr uint32_t ACC_EMPTY_COUNT = 2 * EPI_WARPS;       // epilogue warps of both CTAs
 
 static_assert(SF_COL0 + STAGES * SF_BUF_COLS <= TMEM_COLS, "TMEM budget");
@@ -79,11 +84,10 @@ static_assert(STAGE_BYTES % 1024 == 0, "stage alignment for the 128-byte swizzle
 constexpr uint32_t IDESC = (1u << 7) | (1u << 10) | (uint32_t(PAIR_N >> 3) << 17) | (uint32_t(PAIR_M >> 4) << 24);
 
 struct Smem {
-    uint64_t full[STAGES];      // leader: A and W boxes of both CTAs
+    uint64_t full[STAGES];      // leader: A and W boxes of both CTAs and the stage's scales in TMEM
     uint64_t empty[STAGES];     // each CTA: stage consumed (MMA commit fan-out)
     uint64_t sf_full[SF_SLOTS]; // leader: both CTAs' scale boxes landed
     uint64_t sf_empty[SF_SLOTS];// each CTA: scale slot copied (copier commit fan-out)
-    uint64_t sf_ready[STAGES];  // leader: scales copied into both CTAs' TMEM
     uint64_t acc_full;          // each CTA: accumulator complete (commit fan-out)
     uint64_t acc_empty;         // leader: both CTAs' epilogues drained TMEM
     uint64_t drain;             // leader: every MMA finished before teardown
@@ -157,9 +161,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
-            mbar_init(smem_u32(&sm->full[s]), 2);  // the leader's A and W producers
+            mbar_init(smem_u32(&sm->full[s]), FULL_COUNT);
             mbar_init(smem_u32(&sm->empty[s]), 1);
-            mbar_init(smem_u32(&sm->sf_ready[s]), SF_READY_COUNT);
         }
         for (int j = 0; j < SF_SLOTS; ++j) {
             mbar_init(smem_u32(&sm->sf_full[j]), 1);
@@ -260,8 +263,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                 tc_fence_after();
                 bool ok = true;
                 for (int kt = 0; kt < p.kt_total; ++kt) {
-                    if (!mbar_wait_bounded(smem_u32(&sm->full[stage]), phase, p.wait_limit_ns) ||
-                        !mbar_wait_bounded_cluster(smem_u32(&sm->sf_ready[stage]), phase, p.wait_limit_ns)) {
+                    // codes of both CTAs landed and the stage's scales are in TMEM
+                    if (!mbar_wait_bounded(smem_u32(&sm->full[stage]), phase, p.wait_limit_ns)) {
                         raise_timeout_pair(sm, p.status);
                         ok = false;
                         break;
@@ -316,7 +319,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                     tc_cp_pair_32x128b_x4(sf_t + 16 + kb * 8, smem_desc(sfb_smem(slot) + kb * SF_TILE, 0, 128, 0));
                     tc_cp_pair_32x128b_x4(sf_t + 16 + kb * 8 + 4,
                                           smem_desc(sfb_smem(slot) + p.sf_box_bytes + kb * SF_TILE, 0, 128, 0));
-                    tc_commit_pair(smem_u32(&sm->sf_ready[stage]));
+                    tc_commit_pair(smem_u32(&sm->full[stage]));
                     tc_commit_pair_both(smem_u32(&sm->sf_empty[slot]), 3);  // scale slot free in both CTAs
                     if (++stage == STAGES) {
                         stage = 0;
