@@ -48,17 +48,24 @@ FP4_PER_BF16 = 4.0  # dense FP4 : dense BF16 tensor throughput on B200 (9 : 2.25
 FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # DRAM bytes (read + write) per GEMM launch, mean over the four GEMM launches of
 # one layer, from one ncu capture of this kernel source (profiles/
-# gemm_nvf4_kernel_layer_8192tok.md gives the command).  Reported only while
-# the kernel source still has the captured hash.
-GEMM_TRAFFIC = {"source_sha256_12": "cb4df766954e", "bytes_per_launch": 266.044e6}
-GEMM_SOURCE = os.path.join(ROOT, "nvfp4_w4a4_quantized_act_b200", "csrc", "gemm_kernel.cuh")
+# gemm_nvf4_pair_kernel_layer_8192tok.md gives the command).  Reported only
+# while the kernel sources still have the captured hash.
+GEMM_TRAFFIC = {"source_sha256_12": "aa7977a091bd", "bytes_per_launch": 329.310e6}
+GEMM_SOURCES = [os.path.join(ROOT, "nvfp4_w4a4_quantized_act_b200", "csrc", f)
+                for f in ("gemm_kernel.cuh", "gemm_pair_kernel.cuh", "ptx_sm100.cuh")]
+
+
+def gemm_source_hash():
+    import hashlib
+    h = hashlib.sha256()
+    for path in GEMM_SOURCES:
+        with open(path, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:12]
 
 
 def gemm_traffic():
-    import hashlib
-    with open(GEMM_SOURCE, "rb") as f:
-        h = hashlib.sha256(f.read()).hexdigest()[:12]
-    return GEMM_TRAFFIC["bytes_per_launch"] if h == GEMM_TRAFFIC["source_sha256_12"] else None
+    return GEMM_TRAFFIC["bytes_per_launch"] if gemm_source_hash() == GEMM_TRAFFIC["source_sha256_12"] else None
 
 
 def parse_args():
@@ -360,7 +367,8 @@ def bench_gpu(args, rank, world, local):
             "parallelism": f"replicas x{world} (no collectives)",
         },
         "roofline": {
-            "kernel": "gemm_nvf4_kernel (tcgen05 block-scaled FP4 GEMM; per-module-scale or SwiGLU epilogue)",
+            "kernel": "gemm_nvf4_pair_kernel (CTA-pair tcgen05 block-scaled FP4 GEMM, 256x256 tiles; "
+                      "per-module-scale or SwiGLU epilogue)",
             "bound": "tensor",
             "achieved": round(gemm_tflops, 1),
             "peak": round(fp4_peak, 1),
