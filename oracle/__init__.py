@@ -88,6 +88,12 @@ def _L():
         lib.oracle_linear_sampled.argtypes = [c_p, c_p, c_f, c_p, c_p, c_p, c_i64, c_p, c_p, c_i64, c_p, c_p]
         lib.oracle_swiglu.restype = None
         lib.oracle_swiglu.argtypes = [c_p, c_i64, c_i64, c_i64, c_p]
+        lib.oracle_e4m3_encode.restype = ctypes.c_int
+        lib.oracle_e4m3_encode.argtypes = [c_f]
+        lib.oracle_fp8_kv_scale.restype = c_f
+        lib.oracle_fp8_kv_scale.argtypes = [c_f]
+        lib.oracle_fp8_kv_quantize.restype = None
+        lib.oracle_fp8_kv_quantize.argtypes = [c_p, c_i64, c_i64, c_i64, c_f, c_p, c_i64]
         _lib = lib
     return _lib
 
@@ -295,3 +301,30 @@ def silu_mul(g: np.ndarray, u: np.ndarray) -> np.ndarray:
     """silu(g) * u = g / (1 + exp(-g)) * u, in fp64."""
     g = np.asarray(g, dtype=np.float64)
     return g / (1.0 + np.exp(-g)) * np.asarray(u, dtype=np.float64)
+
+
+# ------------------------------------------------------ FP8 KV-cache codec
+# The KV cache in FP8 (E4M3) with one calibrated FP32 decode scale per cache
+# tensor ("ship the calibrated KV-cache scales": freegardner.com, section
+# "The Calibrated Cache That Ships for Free"; thevalue.engineering, section
+# "Efficiency Gains and Serving Optimization").  Readings: s = amax / 448,
+# code = E4M3_RNE_satfinite(x / s), sign kept.
+
+def e4m3_encode_signed(y: float) -> int:
+    """E4M3 byte of a signed fp32 value: nearest even magnitude, saturating
+    at 448, sign bit from the input (so -0 and small negatives give 0x80)."""
+    return _L().oracle_e4m3_encode(float(np.float32(y)))
+
+
+def fp8_kv_scale(a: float) -> float:
+    """Calibrated FP32 decode scale s = amax / 448 (1.0 when amax == 0)."""
+    return float(np.float32(_L().oracle_fp8_kv_scale(float(np.float32(a)))))
+
+
+def fp8_kv_quantize(x_bits: np.ndarray, s: float) -> np.ndarray:
+    """FP8 codes [rows, cols] (uint8) of a bf16 matrix (uint16 bits)."""
+    x = np.ascontiguousarray(x_bits).view(np.uint16)
+    rows, cols = x.shape
+    out = np.empty((rows, cols), dtype=np.uint8)
+    _L().oracle_fp8_kv_quantize(_ptr(x), rows, cols, cols, float(np.float32(s)), _ptr(out), cols)
+    return out

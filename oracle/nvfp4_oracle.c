@@ -332,3 +332,46 @@ void oracle_swiglu(const uint16_t *gate_up, int64_t rows, int64_t F, int64_t ld,
             h[r * F + j] = oracle_double_to_bf16(s * uv);
         }
 }
+
+/* --------------------------------------------- FP8 KV-cache quantization */
+/*
+ * The attention KV cache in FP8 with a calibrated per-tensor scale: "ship the
+ * calibrated KV-cache scales", which are "performance-free" when calibrated
+ * (freegardner.com, "Quantizing All Layers Reveals Recurrent Memory Is
+ * Robust", section "The Calibrated Cache That Ships for Free";
+ * thevalue.engineering, "NVFP4 W4A4 quantization compresses 27B hybrid
+ * models", section "Efficiency Gains and Serving Optimization"; the
+ * kipquest.com abstract).  The pages give no formula.  Readings: one FP32
+ * decode scale s per cache tensor (x ~= e4m3(code) * s), calibrated as
+ * s = fl32(amax / 448) (1 if amax == 0, as for the NVFP4 global scale), and
+ * code = E4M3_RNE_satfinite(fl32(x / s)) with the sign bit copying the sign
+ * of x, so negative values that round to zero give 0x80.
+ */
+
+/* Signed E4M3: the magnitude by enumeration (oracle_e4m3_encode_nonneg),
+ * the sign bit from the input. */
+int oracle_e4m3_encode(float y)
+{
+    int m = oracle_e4m3_encode_nonneg(fabsf(y));
+    return signbit(y) ? (m | 0x80) : m;
+}
+
+float oracle_fp8_kv_scale(float amax)
+{
+    if (amax == 0.0f)
+        return 1.0f;
+    float s = amax / 448.0f;
+    return s;
+}
+
+/* out[r, c] = E4M3(fl32(x[r, c] / s)) for a row-major bf16 matrix (leading
+ * dimension ld) into a byte matrix with leading dimension ldo. */
+void oracle_fp8_kv_quantize(const uint16_t *x, int64_t rows, int64_t cols, int64_t ld, float s, uint8_t *out,
+                            int64_t ldo)
+{
+    for (int64_t r = 0; r < rows; r++)
+        for (int64_t c = 0; c < cols; c++) {
+            float y = oracle_bf16_to_float(x[r * ld + c]) / s;
+            out[r * ldo + c] = (uint8_t)oracle_e4m3_encode(y);
+        }
+}
