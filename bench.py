@@ -340,6 +340,7 @@ def bench_gpu(args, rank, world, local):
 
     # quantize kernel throughput: one activation [8192, 5120] at HBM roofline
     quant = quantize_roofline(stack, pk, pk_kind)
+    kv = fp8_kv_roofline(pk, pk_kind)
 
     e2e = None
     if not args.no_e2e:
@@ -382,6 +383,7 @@ def bench_gpu(args, rank, world, local):
             "frac_of_datasheet_9pf": round(gemm_tflops / 9000.0, 4),
         },
         "quantize_roofline": quant,
+        "fp8_kv_roofline": kv,
         "gemm_share_of_step": round(sum(gemm_ms) / ms_per_step, 4),
         "gpu_launches": int(launches),
         "clocks": clk,
@@ -424,6 +426,49 @@ def quantize_roofline(stack, pk, pk_kind):
             "bound": "hbm", "achieved": round(gbs, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
             "frac": round(gbs / pk["hbm_gbs"], 4), "us": round(ms * 1e3, 2),
             "algorithmic_bytes": int(alg), "peak_basis": pk_kind, "l2": "256 MB flush before each launch"}
+
+
+def fp8_kv_roofline(pk, pk_kind):
+    """FP8 KV-cache quantization with a calibrated scale, L2 flushed before
+    each launch; 3 bytes per element (bf16 in, one E4M3 byte out).  Two
+    launches shapes: the K cache of one attention layer at 8192 tokens (8 KV
+    heads x 128 = [8192, 1024], what one layer writes), and the K and V caches
+    of all 16 attention layers of the chunk as one [262144, 1024] launch (the
+    roofline figure: the per-layer launch is short enough that launch and
+    ramp-up time are a large part of it)."""
+    from nvfp4_w4a4_quantized_act_b200 import ops
+    from nvfp4_w4a4_quantized_act_b200 import workloads as wl
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+
+    def timed(rows):
+        X = wl.activation_normal(rows, 1024, seed=1024, n_outliers=8, scale=20.0).to("cuda")
+        scale = ops.fp8_kv_calibrate(X)
+        out = torch.empty((rows, 1024), dtype=torch.uint8, device="cuda")
+        ts = []
+        for i in range(13):
+            flush.zero_()
+            s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s.record()
+            ops.fp8_kv_quantize(X, scale, out=out)
+            e.record()
+            e.synchronize()
+            if i >= 3:
+                ts.append(s.elapsed_time(e))
+        del X, out
+        return statistics.median(ts)
+
+    ms_layer = timed(TOKENS)
+    rows_all = TOKENS * 16 * 2
+    ms_all = timed(rows_all)
+    alg = rows_all * 1024 * 3
+    gbs = alg / (ms_all * 1e-3) / 1e9
+    return {"kernel": "kv_quantize_kernel (FP8 E4M3, calibrated per-tensor scale), K+V caches of 16 attention "
+                      "layers at 8192 tokens as one [262144, 1024] bf16 launch",
+            "bound": "hbm", "achieved": round(gbs, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
+            "frac": round(gbs / pk["hbm_gbs"], 4), "us": round(ms_all * 1e3, 2),
+            "algorithmic_bytes": int(alg), "peak_basis": pk_kind, "l2": "256 MB flush before each launch",
+            "one_layer_k_cache_us": round(ms_layer * 1e3, 2),
+            "one_layer_k_cache_gbs": round(TOKENS * 1024 * 3 / (ms_layer * 1e-3) / 1e9, 1)}
 
 
 def bench_e2e(stack, args, world):

@@ -274,6 +274,35 @@ int nvfp4_linear_fused_noalloc(const void *X, int64_t M, int64_t K,
                                const nvfp4_segment *segs, const float *g_w, int nseg,
                                void *out, unsigned flags, void *stream);
 
+/* ------------------------------------------------- FP8 KV-cache (E4M3)
+ *
+ * The attention KV cache in FP8 E4M3 with one calibrated FP32 scale per cache
+ * tensor: the pages' recipe is to "ship the calibrated KV-cache scales",
+ * which they report as performance-free (freegardner.com, "Quantizing All
+ * Layers Reveals Recurrent Memory Is Robust", section "The Calibrated Cache
+ * That Ships for Free"; thevalue.engineering, "NVFP4 W4A4 quantization
+ * compresses 27B hybrid models", section "Efficiency Gains and Serving
+ * Optimization").  The pages give no formula; the reading used here:
+ *   scale s = fl32(amax / 448) (1.0 when amax == 0), a decode multiplier,
+ *   code    = E4M3 round-to-nearest-even, saturating at +-448, of fl32(x / s),
+ *             the sign bit copying the sign of x.
+ * X is bf16 [rows, cols] row-major with leading dimension ldx (elements);
+ * cols % 8 == 0 (NVFP4_ERR_UNSUPPORTED_SHAPE otherwise), X 16-byte aligned
+ * and ldx % 8 == 0 (NVFP4_ERR_MISALIGNED).  Any rows >= 0. */
+
+/* Calibration: *scale (device fp32) = s for X.  ws: device workspace of at
+ * least nvfp4_quant_workspace_bytes(1) bytes (its first word is overwritten).
+ * Non-finite inputs latch NVFP4_ERR_NONFINITE (nvfp4_get_status). */
+int nvfp4_fp8_kv_calibrate(const void *X, int64_t rows, int64_t cols, int64_t ldx, float *scale, void *ws,
+                           size_t ws_bytes, void *stream);
+
+/* Quantization with a calibrated scale: out[r, c] = code of X[r, c], out is
+ * bytes [rows, cols] with leading dimension ldo (8-byte aligned base, ldo % 8
+ * == 0).  scale: device fp32, read by the kernel; if it is not a positive
+ * finite number nothing is written and NVFP4_ERR_NONFINITE is latched. */
+int nvfp4_fp8_kv_quantize(const void *X, int64_t rows, int64_t cols, int64_t ldx, const float *scale, uint8_t *out,
+                          int64_t ldo, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

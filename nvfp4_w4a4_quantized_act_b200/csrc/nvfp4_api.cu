@@ -13,6 +13,7 @@
 #include "nvfp4.h"
 #include "gemm_kernel.cuh"
 #include "gemm_pair_kernel.cuh"
+#include "kv_cache_kernels.cuh"
 #include "quantize_kernels.cuh"
 
 namespace {
@@ -847,4 +848,92 @@ extern "C" int nvfp4_linear_swiglu(const void *X, int64_t M, int64_t K, const ui
         return rc;
     // h -> NVFP4 with the dynamic scale folded in by the epilogue
     return run_quantize_from_amax(d, h, M, F, F, one_seg, h_codes, h_sf, g_h, h_amax, s);
+}
+
+// ------------------------------------------------- FP8 KV-cache (E4M3)
+
+namespace {
+
+int check_kv_shape(const void *X, int64_t rows, int64_t cols, int64_t ldx)
+{
+    if (rows < 0 || cols < 0 || ldx < cols || (rows > 0 && cols > 0 && X == nullptr))
+        return NVFP4_ERR_INVALID_ARG;
+    if (cols % 8 != 0)
+        return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(X) || ldx % 8 != 0)
+        return NVFP4_ERR_MISALIGNED;
+    return NVFP4_OK;
+}
+
+}  // namespace
+
+extern "C" int nvfp4_fp8_kv_calibrate(const void *X, int64_t rows, int64_t cols, int64_t ldx, float *scale, void *ws,
+                                      size_t ws_bytes, void *stream)
+{
+    int rc = check_kv_shape(X, rows, cols, ldx);
+    if (rc != NVFP4_OK)
+        return rc;
+    if (scale == nullptr)
+        return NVFP4_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(scale) & 3u)
+        return NVFP4_ERR_MISALIGNED;
+    if (ws == nullptr || ws_bytes < nvfp4_quant_workspace_bytes(1) || (reinterpret_cast<uintptr_t>(ws) & 3u))
+        return NVFP4_ERR_WORKSPACE;
+    DeviceState *d = device_state();
+    if (d == nullptr)
+        return NVFP4_ERR_CUDA;
+    if (!d->supported)
+        return NVFP4_ERR_NO_DEVICE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint32_t *amax = static_cast<uint32_t *>(ws);
+    if (cudaMemsetAsync(amax, 0, sizeof(uint32_t), s) != cudaSuccess)
+        return NVFP4_ERR_CUDA;
+    g_launches++;
+    if (rows > 0 && cols > 0) {
+        nvfp4::SegRows seg;
+        nvfp4_segment one = {0, rows};
+        check_segments(&one, 1, rows, &seg);
+        const int grid = static_cast<int>(std::min<int64_t>(cdiv(rows, 8), int64_t(d->sm_count) * 8));
+        nvfp4::amax_kernel<<<grid, 256, 0, s>>>(static_cast<const uint16_t *>(X), rows, cols, ldx, seg, amax,
+                                                d->status);
+        g_launches++;
+        if (launch_ok() != NVFP4_OK)
+            return NVFP4_ERR_CUDA;
+    }
+    nvfp4::kv::kv_scale_kernel<<<1, 32, 0, s>>>(amax, scale);
+    g_launches++;
+    return launch_ok();
+}
+
+extern "C" int nvfp4_fp8_kv_quantize(const void *X, int64_t rows, int64_t cols, int64_t ldx, const float *scale,
+                                     uint8_t *out, int64_t ldo, void *stream)
+{
+    int rc = check_kv_shape(X, rows, cols, ldx);
+    if (rc != NVFP4_OK)
+        return rc;
+    if (scale == nullptr || ldo < cols || (rows > 0 && cols > 0 && out == nullptr))
+        return NVFP4_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(scale) & 3u) || (reinterpret_cast<uintptr_t>(out) & 7u) || ldo % 8 != 0)
+        return NVFP4_ERR_MISALIGNED;
+    if (rows == 0 || cols == 0)
+        return NVFP4_OK;
+    DeviceState *d = device_state();
+    if (d == nullptr)
+        return NVFP4_ERR_CUDA;
+    if (!d->supported)
+        return NVFP4_ERR_NO_DEVICE;
+    nvfp4::kv::KvParams p;
+    p.X = static_cast<const uint16_t *>(X);
+    p.ld = ldx;
+    p.rows = rows;
+    p.cols = cols;
+    p.scale = scale;
+    p.out = out;
+    p.ldo = ldo;
+    p.status = d->status;
+    const int64_t groups = rows * (cols / 8);
+    const int grid = static_cast<int>(std::min<int64_t>(cdiv(groups, 256), int64_t(d->sm_count) * 16));
+    nvfp4::kv::kv_quantize_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(p);
+    g_launches++;
+    return launch_ok();
 }

@@ -35,6 +35,7 @@ EXPORTED = [
     "nvfp4_linear", "nvfp4_swiglu_quantize", "nvfp4_get_status", "nvfp4_status_string",
     "nvfp4_device_supported", "nvfp4_launch_count", "nvfp4_linear_fused_noalloc",
     "nvfp4_quantize_weights_gated", "nvfp4_linear_swiglu", "nvfp4_gemm_prequant_swiglu",
+    "nvfp4_fp8_kv_calibrate", "nvfp4_fp8_kv_quantize",
 ]
 
 
@@ -84,6 +85,8 @@ def lib() -> ctypes.CDLL:
         "nvfp4_linear_swiglu": (ctypes.c_int, [vp, i64, i64, u8p, u8p, i64, fp, vp, u8p, u8p, fp, ctypes.c_uint,
                                                vp, sz, vp]),
         "nvfp4_gemm_prequant_swiglu": (ctypes.c_int, [u8p, u8p, fp, i64, i64, u8p, u8p, i64, fp, vp, vp, sz, vp]),
+        "nvfp4_fp8_kv_calibrate": (ctypes.c_int, [vp, i64, i64, i64, fp, vp, sz, vp]),
+        "nvfp4_fp8_kv_quantize": (ctypes.c_int, [vp, i64, i64, i64, fp, u8p, i64, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -368,3 +371,32 @@ def gemm_prequant_swiglu(a_codes, a_sf, g_a, M: int, K: int, w: QuantizedWeight,
                                             _p(w.g_w), _p(h), _p(ws), ws.numel(), _stream(stream)),
            "nvfp4_gemm_prequant_swiglu")
     return h, ws
+
+
+def fp8_kv_calibrate(X: torch.Tensor, scale=None, ws=None, stream=None) -> torch.Tensor:
+    """nvfp4_fp8_kv_calibrate -> the calibrated FP8 KV-cache scale (device
+    fp32 [1]) of a bf16 [rows, cols] cache tensor."""
+    _require_cuda(X)
+    assert X.dtype == torch.bfloat16 and X.dim() == 2 and X.stride(1) == 1
+    rows, cols = X.shape
+    if scale is None:
+        scale = torch.empty(1, dtype=torch.float32, device=X.device)
+    if ws is None:
+        ws = _empty_u8(quant_workspace_bytes(1), X.device)
+    _check(lib().nvfp4_fp8_kv_calibrate(_p(X), rows, cols, X.stride(0), _p(scale), _p(ws), ws.numel(),
+                                        _stream(stream)), "nvfp4_fp8_kv_calibrate")
+    return scale
+
+
+def fp8_kv_quantize(X: torch.Tensor, scale: torch.Tensor, out=None, stream=None) -> torch.Tensor:
+    """nvfp4_fp8_kv_quantize -> E4M3 codes (uint8 [rows, cols]) of a bf16 cache
+    tensor with a calibrated scale (device fp32)."""
+    _require_cuda(X, scale)
+    assert X.dtype == torch.bfloat16 and X.dim() == 2 and X.stride(1) == 1
+    rows, cols = X.shape
+    if out is None:
+        out = torch.empty((rows, cols), dtype=torch.uint8, device=X.device)
+    assert out.dtype == torch.uint8 and out.stride(1) == 1
+    _check(lib().nvfp4_fp8_kv_quantize(_p(X), rows, cols, X.stride(0), _p(scale), _p(out), out.stride(0),
+                                       _stream(stream)), "nvfp4_fp8_kv_quantize")
+    return out

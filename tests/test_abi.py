@@ -86,3 +86,26 @@ def test_argument_errors_return_before_launch(L):
     assert L.nvfp4_swiglu_quantize(fake, 8, 24, 48, fake, fake, fake, fake, fake, 256, None) == 2
     for code in range(9):
         assert ops.status_string(code)
+
+
+def test_fp8_kv_argument_errors_return_before_launch(L):
+    fake = ctypes.c_void_p(1 << 20)  # 16-byte aligned, never dereferenced: checks fail first
+    mis8 = ctypes.c_void_p((1 << 20) + 8)
+    mis4 = ctypes.c_void_p((1 << 20) + 4)
+    # calibrate: cols % 8, ld < cols, null input, null scale, misaligned X, small workspace
+    assert L.nvfp4_fp8_kv_calibrate(fake, 4, 12, 16, fake, fake, 256, None) == 2
+    assert L.nvfp4_fp8_kv_calibrate(fake, 4, 16, 8, fake, fake, 256, None) == 1
+    assert L.nvfp4_fp8_kv_calibrate(None, 4, 16, 16, fake, fake, 256, None) == 1
+    assert L.nvfp4_fp8_kv_calibrate(fake, 4, 16, 16, None, fake, 256, None) == 1
+    assert L.nvfp4_fp8_kv_calibrate(mis8, 4, 16, 16, fake, fake, 256, None) == 3
+    assert L.nvfp4_fp8_kv_calibrate(fake, 4, 16, 20, fake, fake, 256, None) == 3
+    assert L.nvfp4_fp8_kv_calibrate(fake, 4, 16, 16, fake, fake, 2, None) == 7
+    # quantize: same shape rules, plus ldo < cols, misaligned out / ldo
+    assert L.nvfp4_fp8_kv_quantize(fake, 4, 12, 16, fake, fake, 16, None) == 2
+    assert L.nvfp4_fp8_kv_quantize(fake, 4, 16, 16, fake, fake, 8, None) == 1
+    assert L.nvfp4_fp8_kv_quantize(fake, 4, 16, 16, None, fake, 16, None) == 1
+    assert L.nvfp4_fp8_kv_quantize(fake, 4, 16, 16, fake, None, 16, None) == 1
+    assert L.nvfp4_fp8_kv_quantize(fake, 4, 16, 16, fake, mis4, 16, None) == 3
+    assert L.nvfp4_fp8_kv_quantize(fake, 4, 16, 16, fake, fake, 20, None) == 3
+    # empty tensors are no-ops
+    assert L.nvfp4_fp8_kv_quantize(None, 0, 16, 16, fake, None, 16, None) == 0
