@@ -104,8 +104,12 @@ size_t nvfp4_sf_bytes(int64_t rows, int64_t K);
 size_t nvfp4_quant_workspace_bytes(int nseg);
 
 /* Workspace bytes needed by nvfp4_linear / nvfp4_linear_fused for an [M, K]
- * input: the quantized activation (codes and scale factors), its amax and
- * global scale.  N and nseg do not change the size and may be 0. */
+ * input and N outputs: the quantized activation (codes and scale factors),
+ * its amax and global scale and, for M <= 128 (decode-sized inputs), the
+ * fp32 partial sums of the split-K GEMM (splits x M x N x 4 bytes, at most 8
+ * splits; the split count depends on M, N and K only, so results do not
+ * depend on the device).  nseg does not change the size and may be 0.  With
+ * N = 0 the size covers the activation only, enough for every M > 128. */
 size_t nvfp4_workspace_bytes(int64_t M, int64_t N, int64_t K, int nseg);
 
 /* Offline weight quantization (post-training, per module).

@@ -76,6 +76,13 @@ struct Params {
     int32_t M, N, K;
     int32_t num_m, num_n, num_tiles;
     int32_t pair_m, pair_n, pair_tiles;  // 256 x 256 tiles of the CTA-pair kernel
+    // Split-K (single-CTA kernel, small M): work item t covers tile
+    // t % num_tiles over the K steps of split t / num_tiles; with splits > 1
+    // the epilogue writes alpha * acc as fp32 to partial[split][M][N] and a
+    // finalize kernel sums the splits in order.
+    int32_t splits;
+    int32_t kt_per_split;
+    float *partial;
     int32_t kb_total;    // K / 64
     int32_t kt_total;    // ceil(kb_total / 4)
     int32_t n_row_tiles; // ceil(N / 128): scale tiles of W per K-step
@@ -117,6 +124,14 @@ __device__ __forceinline__ void tile_coords(const Params &p, int tile, int &m_bl
         m_blk = tile % p.num_m;
         n_blk = tile / p.num_m;
     }
+}
+
+__device__ __forceinline__ void work_item(const Params &p, int item, int &tile, int &split, int &kt0, int &kt1)
+{
+    split = item / p.num_tiles;
+    tile = item - split * p.num_tiles;
+    kt0 = split * p.kt_per_split;
+    kt1 = min(kt0 + p.kt_per_split, p.kt_total);
 }
 
 struct Smem {
@@ -211,6 +226,46 @@ __device__ __forceinline__ void store_64(const Params &p, const float *alpha, in
     }
 }
 
+// Split-K partial: alpha * acc for 64 columns of one row, fp32, into the
+// split's [M, N] slice of p.partial.
+__device__ __forceinline__ void store_partial_64(const Params &p, int split, const float *alpha, int32_t row,
+                                                 int32_t col0, const uint32_t (&v)[64])
+{
+    if (row >= p.M || col0 >= p.N)
+        return;
+    float *o = p.partial + (static_cast<int64_t>(split) * p.M + row) * p.N + col0;
+    if ((p.N & 3) == 0 && col0 + 64 <= p.N) {
+#pragma unroll
+        for (int j = 0; j < 64; j += 4) {
+            const float4 a = *reinterpret_cast<const float4 *>(&alpha[j]);
+            *reinterpret_cast<float4 *>(o + j) =
+                make_float4(__fmul_rn(__uint_as_float(v[j]), a.x), __fmul_rn(__uint_as_float(v[j + 1]), a.y),
+                            __fmul_rn(__uint_as_float(v[j + 2]), a.z), __fmul_rn(__uint_as_float(v[j + 3]), a.w));
+        }
+    } else {
+        for (int j = 0; j < 64 && col0 + j < p.N; ++j)
+            o[j] = __fmul_rn(__uint_as_float(v[j]), alpha[j]);
+    }
+}
+
+// out[m, n] = round( sum over splits s = 0, 1, ... of partial[s][m][n] ), the
+// splits added in order (deterministic), bf16 round-to-nearest-even or fp32.
+__global__ void __launch_bounds__(256) splitk_finalize_kernel(const float *__restrict__ partial, int32_t splits,
+                                                              int64_t M, int64_t N, void *out, int32_t out_fp32)
+{
+    const int64_t total = M * N;
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total; i += stride) {
+        float acc = partial[i];
+        for (int s = 1; s < splits; ++s)
+            acc = __fadd_rn(acc, partial[static_cast<int64_t>(s) * total + i]);
+        if (out_fp32)
+            static_cast<float *>(out)[i] = acc;
+        else
+            static_cast<__nv_bfloat16 *>(out)[i] = __float2bfloat16_rn(acc);
+    }
+}
+
 // Store 128 bf16 values of one row (as 64 packed pairs) at [row, col0).
 __device__ __forceinline__ void store_bf16_packed_128(const Params &p, int32_t row, int32_t col0,
                                                       const uint32_t (&pk)[64])
@@ -293,12 +348,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (lane == 0 && !p.inject_stall) {
             int stage = 0;
             uint32_t phase = 0;
-            for (int tile = blockIdx.x; tile < p.num_tiles && !sm->abort_flag; tile += gridDim.x) {
-                int m_blk, n_blk;
+            for (int item = blockIdx.x; item < p.num_tiles * p.splits && !sm->abort_flag; item += gridDim.x) {
+                int tile, split, kt0, kt1, m_blk, n_blk;
+                work_item(p, item, tile, split, kt0, kt1);
                 tile_coords(p, tile, m_blk, n_blk);
                 const int m0 = m_blk * BM, n0 = n_blk * BN;
                 const int rb0 = n0 >> 7;  // first 128-row scale tile of W
-                for (int kt = 0; kt < p.kt_total; ++kt) {
+                for (int kt = kt0; kt < kt1; ++kt) {
                     if (!mbar_wait_bounded(smem_u32(&sm->empty[stage]), phase ^ 1u, p.wait_limit_ns)) {
                         raise_timeout(sm, p.status);
                         break;
@@ -332,14 +388,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             int stage = 0;
             uint32_t phase = 0;
             int local = 0;
-            for (int tile = blockIdx.x; tile < p.num_tiles && !sm->abort_flag; tile += gridDim.x, ++local) {
+            for (int item = blockIdx.x; item < p.num_tiles * p.splits && !sm->abort_flag;
+                 item += gridDim.x, ++local) {
+                int tile, split, kt0, kt1;
+                work_item(p, item, tile, split, kt0, kt1);
                 if (!mbar_wait_bounded(smem_u32(&sm->acc_empty), (local & 1) ^ 1u, p.wait_limit_ns)) {
                     raise_timeout(sm, p.status);
                     break;
                 }
                 tc_fence_after();
                 bool ok = true;
-                for (int kt = 0; kt < p.kt_total; ++kt) {
+                for (int kt = kt0; kt < kt1; ++kt) {
                     if (!mbar_wait_bounded(smem_u32(&sm->full[stage]), phase, p.wait_limit_ns) ||
                         !mbar_wait_bounded(smem_u32(&sm->sf_ready[stage]), phase, p.wait_limit_ns)) {
                         raise_timeout(sm, p.status);
@@ -352,7 +411,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     const uint32_t sfb_t = sfa_t + 4 * KB_PER_STAGE;
                     for (int kb = 0; kb < nkb; ++kb) {
                         const uint64_t adesc = smem_desc(a_smem(stage) + kb * 32, 16, 1024, 2);
-                        const uint32_t acc_flag = (kt > 0 || kb > 0) ? 1u : 0u;
+                        const uint32_t acc_flag = (kt > kt0 || kb > 0) ? 1u : 0u;
 #pragma unroll
                         for (int h = 0; h < 2; ++h) {
                             const uint64_t bdesc =
@@ -381,9 +440,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (lane == 0) {
             int stage = 0;
             uint32_t phase = 0;
-            for (int tile = blockIdx.x; tile < p.num_tiles && !sm->abort_flag; tile += gridDim.x) {
+            for (int item = blockIdx.x; item < p.num_tiles * p.splits && !sm->abort_flag; item += gridDim.x) {
+                int tile, split, kt0, kt1;
+                work_item(p, item, tile, split, kt0, kt1);
                 bool ok = true;
-                for (int kt = 0; kt < p.kt_total; ++kt) {
+                for (int kt = kt0; kt < kt1; ++kt) {
                     // The stage's TMEM scale buffer is free: the producer only refilled this
                     // stage after the MMAs that read the buffer last time had completed.
                     if (!mbar_wait_bounded(smem_u32(&sm->full[stage]), phase, p.wait_limit_ns)) {
@@ -422,8 +483,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const float a_up = __fmul_rn(ga, __ldg(p.g_w + 1));
         uint32_t hmax = 0;
         int local = 0;
-        for (int tile = blockIdx.x; tile < p.num_tiles && !sm->abort_flag; tile += gridDim.x, ++local) {
-            int m_blk, n_blk;
+        for (int item = blockIdx.x; item < p.num_tiles * p.splits && !sm->abort_flag; item += gridDim.x, ++local) {
+            int tile, split, kt0, kt1, m_blk, n_blk;
+            work_item(p, item, tile, split, kt0, kt1);  // the gated path never splits K
             tile_coords(p, tile, m_blk, n_blk);
             const int m0 = m_blk * BM, n0 = n_blk * BN;
             const bool ok = mbar_wait_bounded(smem_u32(&sm->acc_full), local & 1, p.wait_limit_ns);
@@ -486,8 +548,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         float *alpha = sm->alpha[warp - EPI_WARP0];
         const float ga = __ldg(p.g_a);
         int local = 0;
-        for (int tile = blockIdx.x; tile < p.num_tiles && !sm->abort_flag; tile += gridDim.x, ++local) {
-            int m_blk, n_blk;
+        for (int item = blockIdx.x; item < p.num_tiles * p.splits && !sm->abort_flag; item += gridDim.x, ++local) {
+            int tile, split, kt0, kt1, m_blk, n_blk;
+            work_item(p, item, tile, split, kt0, kt1);
             tile_coords(p, tile, m_blk, n_blk);
             const int m0 = m_blk * BM, n0 = n_blk * BN;
             __syncwarp();  // this warp's reads of the previous tile's alpha are done
@@ -513,8 +576,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             if (lane == 0)
                 mbar_arrive(smem_u32(&sm->acc_empty));
             const int row = m0 + q * 32 + lane;
-            store_64(p, alpha, row, n0 + hc * HALF_N, v0);
-            store_64(p, alpha + 64, row, n0 + hc * HALF_N + 64, v1);
+            if (p.splits > 1) {
+                store_partial_64(p, split, alpha, row, n0 + hc * HALF_N, v0);
+                store_partial_64(p, split, alpha + 64, row, n0 + hc * HALF_N + 64, v1);
+            } else {
+                store_64(p, alpha, row, n0 + hc * HALF_N, v0);
+                store_64(p, alpha + 64, row, n0 + hc * HALF_N + 64, v1);
+            }
         }
     }
 

@@ -2,6 +2,7 @@
 // carving, TMA descriptor set-up and kernel launches for the NVFP4 W4A4
 // linear layer.  Every entry point is declared and documented in
 // include/nvfp4.h.
+#include <algorithm>
 #include <atomic>
 #include <cstdint>
 #include <cstring>
@@ -239,11 +240,34 @@ int make_out_map(CUtensorMap *map, void *out, int64_t rows, int64_t cols)
     return r == CUDA_SUCCESS ? NVFP4_OK : NVFP4_ERR_CUDA;
 }
 
+// Split-K for small M (one 128-row block): the single-CTA kernel has only
+// cdiv(N, 256) output tiles there, too few to occupy 148 SMs, so each tile's
+// K steps are divided into `splits` contiguous ranges that run as separate
+// work items.  The count depends on the shape alone (sized for 148 SMs), so
+// the result's bits do not depend on the device; every range is non-empty.
+constexpr int kSplitKMax = 8;
+constexpr int kSplitKSms = 148;
+
+int splitk_count(int64_t M, int64_t N, int64_t K)
+{
+    using namespace nvfp4::gemm;
+    if (M <= 0 || M > BM || N <= 0 || K <= 0)
+        return 1;
+    const int64_t tiles = cdiv(N, BN);
+    const int64_t kt_total = cdiv(K / 64, KB_PER_STAGE);
+    const int64_t want = std::min<int64_t>({kSplitKMax, kt_total, std::max<int64_t>(1, kSplitKSms / tiles)});
+    const int64_t kps = cdiv(kt_total, want);
+    return static_cast<int>(cdiv(kt_total, kps));
+}
+
 // h_amax != nullptr selects the gated MLP epilogue (W is [gate | up]
-// interleaved in 128-row blocks, N = 2F, out = h [M, F] bf16).
+// interleaved in 128-row blocks, N = 2F, out = h [M, F] bf16).  partial !=
+// nullptr (room for splitk_count(M, N, K) fp32 [M, N] slices) lets a plain
+// GEMM with M <= 128 split K; the splits are then summed in order by a
+// second kernel.
 int run_gemm(DeviceState *d, const uint8_t *a_codes, const uint8_t *a_sf, const float *g_a, int64_t M, int64_t K,
              const uint8_t *w_codes, const uint8_t *w_sf, int64_t N, const nvfp4::SegRows &seg, const float *g_w,
-             void *out, unsigned flags, cudaStream_t stream, uint32_t *h_amax = nullptr)
+             void *out, unsigned flags, cudaStream_t stream, uint32_t *h_amax = nullptr, float *partial = nullptr)
 {
     using namespace nvfp4::gemm;
     if (M == 0 || N == 0)
@@ -276,6 +300,16 @@ int run_gemm(DeviceState *d, const uint8_t *a_codes, const uint8_t *a_sf, const 
     p.pair_tiles = p.pair_m * p.pair_n;
     p.kb_total = static_cast<int32_t>(K / 64);
     p.kt_total = static_cast<int32_t>(cdiv(K / 64, KB_PER_STAGE));
+    p.splits = 1;
+    p.kt_per_split = p.kt_total;
+    if (partial != nullptr && h_amax == nullptr && !use_pair) {
+        const int S = splitk_count(M, N, K);
+        if (S > 1) {
+            p.splits = S;
+            p.kt_per_split = static_cast<int32_t>(cdiv(p.kt_total, S));
+            p.partial = partial;
+        }
+    }
     p.n_row_tiles = static_cast<int32_t>(n_row_tiles);
     p.sf_box_bytes = sf_box;
     p.sfb_box_rows = sfb_rows;
@@ -319,11 +353,20 @@ int run_gemm(DeviceState *d, const uint8_t *a_codes, const uint8_t *a_sf, const 
             pair::gemm_nvf4_pair_kernel<false><<<grid, pair::NUM_THREADS, pair::SMEM_BYTES, stream>>>(
                 tmA, tmB, tmSFA, tmSFB, tmOut, p);
     } else {
-        const int grid = static_cast<int>(std::min<int64_t>(p.num_tiles, d->sm_count));
+        const int grid = static_cast<int>(std::min<int64_t>(static_cast<int64_t>(p.num_tiles) * p.splits, d->sm_count));
         if (h_amax != nullptr)
             gemm_nvf4_kernel<true><<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(tmA, tmB, tmSFA, tmSFB, p);
         else
             gemm_nvf4_kernel<false><<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(tmA, tmB, tmSFA, tmSFB, p);
+        if (p.splits > 1) {
+            g_launches++;
+            const int rc = launch_ok();
+            if (rc != NVFP4_OK)
+                return rc;
+            const int64_t total = M * N;
+            const int fin_grid = static_cast<int>(std::min<int64_t>(cdiv(total, 256), 4LL * d->sm_count));
+            splitk_finalize_kernel<<<fin_grid, 256, 0, stream>>>(partial, p.splits, M, N, out, p.out_fp32);
+        }
     }
     g_launches++;
     return launch_ok();
@@ -352,6 +395,18 @@ size_t linear_sf_off(int64_t M, int64_t K)
     return static_cast<size_t>(round_up(static_cast<int64_t>(kLinCodesOff + linear_codes_bytes(M, K)), 1024));
 }
 
+// Split-K partial sums follow the activation's scale factors.
+size_t linear_partial_off(int64_t M, int64_t K)
+{
+    return static_cast<size_t>(round_up(static_cast<int64_t>(linear_sf_off(M, K)) + sf_bytes_i(M, K), 256));
+}
+
+size_t linear_partial_bytes(int64_t M, int64_t N, int64_t K)
+{
+    const int S = splitk_count(M, N, K);
+    return S > 1 ? static_cast<size_t>(S) * static_cast<size_t>(M) * static_cast<size_t>(N) * 4 : 0;
+}
+
 }  // namespace
 
 // ======================================================================== C ABI
@@ -374,10 +429,12 @@ size_t nvfp4_quant_workspace_bytes(int nseg)
 
 size_t nvfp4_workspace_bytes(int64_t M, int64_t N, int64_t K, int nseg)
 {
-    (void)N;
     (void)nseg;
-    if (M < 0 || K <= 0 || K % 16 != 0)
+    if (M < 0 || N < 0 || K <= 0 || K % 16 != 0)
         return 0;
+    const size_t partial = linear_partial_bytes(M, N, K);
+    if (partial > 0)
+        return linear_partial_off(M, K) + partial;
     return linear_sf_off(M, K) + static_cast<size_t>(sf_bytes_i(M, K));
 }
 
@@ -526,7 +583,9 @@ int nvfp4_linear_fused(const void *X, int64_t M, int64_t K, const uint8_t *w_cod
     rc = run_quantize(d, X, M, K, K, one_seg, a_codes, a_sf, g_a, g_a, dynamic, amax, s);
     if (rc != NVFP4_OK)
         return rc;
-    return run_gemm(d, a_codes, a_sf, g_a, M, K, w_codes, w_sf, N, seg, g_w, out, flags, s);
+    float *partial =
+        linear_partial_bytes(M, N, K) > 0 ? reinterpret_cast<float *>(base + linear_partial_off(M, K)) : nullptr;
+    return run_gemm(d, a_codes, a_sf, g_a, M, K, w_codes, w_sf, N, seg, g_w, out, flags, s, nullptr, partial);
 }
 
 int nvfp4_linear(const void *X, int64_t M, int64_t K, const uint8_t *w_codes, const uint8_t *w_sf, const float *g_w,

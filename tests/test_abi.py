@@ -45,6 +45,32 @@ def test_sizes(L):
     assert ops.act_scale_offset() == 256
 
 
+def _act_bytes(M, K):
+    codes_end = 1024 + M * K // 2
+    sf_off = -(-codes_end // 1024) * 1024
+    return sf_off + ops.sf_bytes(M, K)
+
+
+@pytest.mark.parametrize("M,N,K,splits", [
+    (16, 5120, 5120, 7),     # 20 tiles of 256 columns, 20 stages: 7 splits of <= 3 stages
+    (1, 1024, 5120, 7),      # 4 tiles: at most 8 splits, 20 stages -> 7 of <= 3
+    (128, 1280, 17408, 8),   # 68 stages: 8 splits of <= 9
+    (64, 16480, 5120, 2),    # 65 tiles: 148 // 65 = 2
+    (128, 34816, 5120, 1),   # 136 tiles fill the GPU: no split
+    (16, 5120, 256, 1),      # one stage of K: no split
+    (129, 5120, 5120, 1),    # more than one 128-row block: CTA-pair GEMM, no split
+])
+def test_decode_workspace_holds_split_partials(L, M, N, K, splits):
+    """M <= 128 linears reserve splits x M x N fp32 partial sums after the
+    activation (256-byte aligned); N = 0 sizes the activation alone."""
+    act = _act_bytes(M, K)
+    assert ops.workspace_bytes(M, 0, K) == act
+    if splits == 1:
+        assert ops.workspace_bytes(M, N, K) == act
+    else:
+        assert ops.workspace_bytes(M, N, K) == -(-act // 256) * 256 + splits * M * N * 4
+
+
 def _segarr(pairs):
     return (ops.Segment * len(pairs))(*[ops.Segment(a, b) for a, b in pairs])
 
@@ -80,6 +106,10 @@ def test_argument_errors_return_before_launch(L):
     assert L.nvfp4_gemm_prequant(fake, fake, fake, -1, 128, fake, fake, 32, segs_ok, fake, 2, fake, 0, None) == 1
     # linear_fused: workspace too small
     assert L.nvfp4_linear_fused(fake, 8, 128, fake, fake, 32, segs_ok, fake, 2, fake, 0, fake, 16, None) == 7
+    # decode-sized linear given only the activation's share (no room for the split-K partials)
+    one = _segarr([(0, 5120)])
+    act_only = ops.workspace_bytes(16, 0, 5120)
+    assert L.nvfp4_linear_fused(fake, 16, 5120, fake, fake, 5120, one, fake, 1, fake, 0, fake, act_only, None) == 7
     # weights: misaligned leading dimension
     assert L.nvfp4_quantize_weights(fake, 32, 64, 68, segs_ok, 2, fake, fake, fake, fake, 256, None) == 3
     # SwiGLU: F % 16
