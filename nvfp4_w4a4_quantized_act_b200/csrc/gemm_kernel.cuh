@@ -253,6 +253,8 @@ __device__ __forceinline__ void store_partial_64(const Params &p, int split, con
 __global__ void __launch_bounds__(256) splitk_finalize_kernel(const float *__restrict__ partial, int32_t splits,
                                                               int64_t M, int64_t N, void *out, int32_t out_fp32)
 {
+    grid_dep_wait();
+    grid_dep_launch_dependents();
     const int64_t total = M * N;
     const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
     for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total; i += stride) {
@@ -336,6 +338,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = sm->tmem_base;
+    // set-up above touches no global memory; from here on the previous
+    // kernel's outputs (the quantized activation) are read
+    grid_dep_wait();
+    grid_dep_launch_dependents();
 
     if (warp == 0 || warp == 3) {
         // ----------------------------------------------------- producers

@@ -193,6 +193,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
     tc_fence_before();
     cluster_sync_all();
     tc_fence_after();
+    // set-up above touches no global memory
+    grid_dep_wait();
+    grid_dep_launch_dependents();
     const uint32_t tmem = sm->tmem_base;
     auto leader_bar = [&](uint64_t *b) { return mapa_shared(smem_u32(b), 0); };
 

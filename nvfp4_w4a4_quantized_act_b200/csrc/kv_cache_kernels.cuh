@@ -25,6 +25,8 @@ namespace kv {
 // s = fl32(amax / 448) (1 when amax == 0) from the amax pass's bf16 bits.
 __global__ void kv_scale_kernel(const uint32_t *__restrict__ amax_bits, float *__restrict__ scale)
 {
+    grid_dep_wait();
+    grid_dep_launch_dependents();
     if (blockIdx.x == 0 && threadIdx.x == 0) {
         const float a = __uint_as_float(amax_bits[0] << 16);
         scale[0] = (a == 0.0f) ? 1.0f : __fdiv_rn(a, 448.0f);
@@ -55,6 +57,8 @@ struct KvParams {
 // conversions, one 8-byte store.
 __global__ void __launch_bounds__(256) kv_quantize_kernel(const KvParams p)
 {
+    grid_dep_wait();
+    grid_dep_launch_dependents();
     const float s = __ldg(p.scale);
     if (!(s > 0.0f) || !(s <= 3.40282347e38f)) {
         // a scale that is not a positive finite number: nothing is written

@@ -112,14 +112,59 @@ int check_segments(const nvfp4_segment *segs, int nseg, int64_t N, nvfp4::SegRow
     return expect == N ? NVFP4_OK : NVFP4_ERR_INVALID_ARG;
 }
 
+thread_local bool t_launch_failed = false;
+
+// Launches a kernel with programmatic stream serialization: the kernel may
+// be scheduled while the previous kernel on the stream is still running and
+// waits for it (griddepcontrol.wait) before touching global memory.  Every
+// kernel of this library does that wait first, so stream order holds.
+template <typename... KArgs, typename... Args>
+void launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream, Args... args)
+{
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kernel, args...) != cudaSuccess)
+        t_launch_failed = true;
+}
+
 int launch_ok()
 {
-    return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
+    const bool failed = t_launch_failed;
+    t_launch_failed = false;
+    return (cudaGetLastError() == cudaSuccess && !failed) ? NVFP4_OK : NVFP4_ERR_CUDA;
+}
+
+// Clears `n` amax words on the stream (a kernel, so that the launches around
+// it keep their programmatic dependencies).
+int zero_words(uint32_t *words, int n, cudaStream_t stream)
+{
+    launch(nvfp4::zero_words_kernel, dim3(1), dim3(32), 0, stream, words, static_cast<int32_t>(n));
+    g_launches++;
+    return launch_ok();
 }
 
 // K1 + K2 for `rows` x K bf16 rows, segment table `seg`.  mode 0: dynamic
 // scale from max|x| (amax words in ws, g written to g_out); mode 1: scale
 // read from g_in.
+//
+// Rows of the amax pass are cut into ranges of 128 16-byte chunks (one
+// four-load sweep of a warp) while rows are too few to give every SM work.
+int64_t amax_slices(int64_t rows, int64_t cols)
+{
+    if (rows >= 1024)
+        return 1;
+    return std::max<int64_t>(1, cdiv(cols >> 3, 128));
+}
+
 int run_quantize(DeviceState *d, const void *X, int64_t rows, int64_t K, int64_t ld, const nvfp4::SegRows &seg,
                  uint8_t *codes, uint8_t *sf, const float *g_in, float *g_out, bool dynamic, uint32_t *amax_ws,
                  cudaStream_t stream, int64_t gate_up_F = 0)
@@ -129,14 +174,14 @@ int run_quantize(DeviceState *d, const void *X, int64_t rows, int64_t K, int64_t
     if (rows_pad * groups * 4 >= (int64_t(1) << 31) || K > (int64_t(1) << 30))
         return NVFP4_ERR_UNSUPPORTED_SHAPE;
     if (dynamic) {
-        if (cudaMemsetAsync(amax_ws, 0, sizeof(uint32_t) * seg.nseg, stream) != cudaSuccess)
+        if (zero_words(amax_ws, seg.nseg, stream) != NVFP4_OK)
             return NVFP4_ERR_CUDA;
-        g_launches++;
         if (rows > 0) {
-            const int64_t warps_needed = rows;
+            const int64_t slices = amax_slices(rows, K);
+            const int64_t warps_needed = rows * slices;
             int grid = static_cast<int>(std::min<int64_t>(cdiv(warps_needed, 8), int64_t(d->sm_count) * 8));
-            nvfp4::amax_kernel<<<grid, 256, 0, stream>>>(static_cast<const uint16_t *>(X), rows, K, ld, seg,
-                                                          amax_ws, d->status);
+            launch(nvfp4::amax_kernel, dim3(grid), dim3(256), 0, stream, static_cast<const uint16_t *>(X), rows, K, ld,
+                   slices, seg, amax_ws, d->status);
             g_launches++;
             if (launch_ok() != NVFP4_OK)
                 return NVFP4_ERR_CUDA;
@@ -159,7 +204,7 @@ int run_quantize(DeviceState *d, const void *X, int64_t rows, int64_t K, int64_t
     p.gate_up_F = static_cast<int32_t>(gate_up_F);
     const int64_t threads = rows_pad * groups * 4;
     int grid = static_cast<int>(std::min<int64_t>(std::max<int64_t>(cdiv(threads, 256), 1), int64_t(d->sm_count) * 16));
-    nvfp4::quantize_kernel<<<grid, 256, 0, stream>>>(p);
+    launch(nvfp4::quantize_kernel, dim3(grid), dim3(256), 0, stream, p);
     g_launches++;
     return launch_ok();
 }
@@ -190,7 +235,7 @@ int run_quantize_from_amax(DeviceState *d, const void *X, int64_t rows, int64_t 
     p.gate_up_F = 0;
     const int64_t threads = rows_pad * groups * 4;
     const int grid = static_cast<int>(std::min<int64_t>(std::max<int64_t>(cdiv(threads, 256), 1), int64_t(d->sm_count) * 16));
-    nvfp4::quantize_kernel<<<grid, 256, 0, stream>>>(p);
+    launch(nvfp4::quantize_kernel, dim3(grid), dim3(256), 0, stream, p);
     g_launches++;
     return launch_ok();
 }
@@ -347,17 +392,17 @@ int run_gemm(DeviceState *d, const uint8_t *a_codes, const uint8_t *a_sf, const 
         // one cluster of two CTAs per pair of SMs, persistent over the pair tiles
         const int grid = 2 * static_cast<int>(std::min<int64_t>(p.pair_tiles, d->sm_count / 2));
         if (h_amax != nullptr)
-            pair::gemm_nvf4_pair_kernel<true><<<grid, pair::NUM_THREADS, pair::SMEM_BYTES, stream>>>(
-                tmA, tmB, tmSFA, tmSFB, tmOut, p);
+            launch(pair::gemm_nvf4_pair_kernel<true>, dim3(grid), dim3(pair::NUM_THREADS), pair::SMEM_BYTES, stream,
+                   tmA, tmB, tmSFA, tmSFB, tmOut, p);
         else
-            pair::gemm_nvf4_pair_kernel<false><<<grid, pair::NUM_THREADS, pair::SMEM_BYTES, stream>>>(
-                tmA, tmB, tmSFA, tmSFB, tmOut, p);
+            launch(pair::gemm_nvf4_pair_kernel<false>, dim3(grid), dim3(pair::NUM_THREADS), pair::SMEM_BYTES, stream,
+                   tmA, tmB, tmSFA, tmSFB, tmOut, p);
     } else {
         const int grid = static_cast<int>(std::min<int64_t>(static_cast<int64_t>(p.num_tiles) * p.splits, d->sm_count));
         if (h_amax != nullptr)
-            gemm_nvf4_kernel<true><<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(tmA, tmB, tmSFA, tmSFB, p);
+            launch(gemm_nvf4_kernel<true>, dim3(grid), dim3(NUM_THREADS), SMEM_BYTES, stream, tmA, tmB, tmSFA, tmSFB, p);
         else
-            gemm_nvf4_kernel<false><<<grid, NUM_THREADS, SMEM_BYTES, stream>>>(tmA, tmB, tmSFA, tmSFB, p);
+            launch(gemm_nvf4_kernel<false>, dim3(grid), dim3(NUM_THREADS), SMEM_BYTES, stream, tmA, tmB, tmSFA, tmSFB, p);
         if (p.splits > 1) {
             g_launches++;
             const int rc = launch_ok();
@@ -365,7 +410,8 @@ int run_gemm(DeviceState *d, const uint8_t *a_codes, const uint8_t *a_sf, const 
                 return rc;
             const int64_t total = M * N;
             const int fin_grid = static_cast<int>(std::min<int64_t>(cdiv(total, 256), 4LL * d->sm_count));
-            splitk_finalize_kernel<<<fin_grid, 256, 0, stream>>>(partial, p.splits, M, N, out, p.out_fp32);
+            launch(splitk_finalize_kernel, dim3(fin_grid), dim3(256), 0, stream, static_cast<const float *>(partial),
+                   p.splits, M, N, out, p.out_fp32);
         }
     }
     g_launches++;
@@ -619,15 +665,13 @@ int nvfp4_swiglu_quantize(const void *gate_up, int64_t M, int64_t F, int64_t ld,
         return NVFP4_ERR_NO_DEVICE;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     uint32_t *amax = static_cast<uint32_t *>(ws);
-    if (cudaMemsetAsync(amax, 0, sizeof(uint32_t), s) != cudaSuccess)
+    if (zero_words(amax, 1, s) != NVFP4_OK)
         return NVFP4_ERR_CUDA;
-    g_launches++;
     if (M > 0) {
         const int64_t threads = M * (F / 8);
         const int grid = static_cast<int>(std::min<int64_t>(cdiv(threads, 256), int64_t(d->sm_count) * 16));
-        nvfp4::swiglu_kernel<<<grid, 256, 0, s>>>(static_cast<const uint16_t *>(gate_up), ld,
-                                                  static_cast<int32_t>(M), static_cast<int32_t>(F),
-                                                  static_cast<uint16_t *>(h), amax);
+        launch(nvfp4::swiglu_kernel, dim3(grid), dim3(256), 0, s, static_cast<const uint16_t *>(gate_up), ld,
+               static_cast<int32_t>(M), static_cast<int32_t>(F), static_cast<uint16_t *>(h), amax);
         g_launches++;
         if (launch_ok() != NVFP4_OK)
             return NVFP4_ERR_CUDA;
@@ -657,7 +701,7 @@ int nvfp4_swiglu_quantize(const void *gate_up, int64_t M, int64_t F, int64_t ld,
     p.gate_up_F = 0;
     const int64_t threads = rows_pad * groups * 4;
     const int grid = static_cast<int>(std::min<int64_t>(std::max<int64_t>(cdiv(threads, 256), 1), int64_t(d->sm_count) * 16));
-    nvfp4::quantize_kernel<<<grid, 256, 0, s>>>(p);
+    launch(nvfp4::quantize_kernel, dim3(grid), dim3(256), 0, s, p);
     g_launches++;
     return launch_ok();
 }
@@ -845,9 +889,8 @@ extern "C" int nvfp4_gemm_prequant_swiglu(const uint8_t *a_codes, const uint8_t 
         return NVFP4_ERR_NO_DEVICE;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     uint32_t *h_amax = static_cast<uint32_t *>(ws);
-    if (cudaMemsetAsync(h_amax, 0, sizeof(uint32_t), s) != cudaSuccess)
+    if (zero_words(h_amax, 1, s) != NVFP4_OK)
         return NVFP4_ERR_CUDA;
-    g_launches++;
     nvfp4::SegRows gu;
     const nvfp4_segment two[2] = {{0, F}, {F, 2 * F}};
     check_segments(two, 2, 2 * F, &gu);
@@ -896,9 +939,8 @@ extern "C" int nvfp4_linear_swiglu(const void *X, int64_t M, int64_t K, const ui
     if (rc != NVFP4_OK)
         return rc;
     // gate/up GEMM with the SwiGLU epilogue -> h (bf16) and max|h|
-    if (cudaMemsetAsync(h_amax, 0, sizeof(uint32_t), s) != cudaSuccess)
+    if (zero_words(h_amax, 1, s) != NVFP4_OK)
         return NVFP4_ERR_CUDA;
-    g_launches++;
     nvfp4::SegRows gu;
     const nvfp4_segment two[2] = {{0, F}, {F, 2 * F}};
     check_segments(two, 2, 2 * F, &gu);
@@ -945,21 +987,21 @@ extern "C" int nvfp4_fp8_kv_calibrate(const void *X, int64_t rows, int64_t cols,
         return NVFP4_ERR_NO_DEVICE;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     uint32_t *amax = static_cast<uint32_t *>(ws);
-    if (cudaMemsetAsync(amax, 0, sizeof(uint32_t), s) != cudaSuccess)
+    if (zero_words(amax, 1, s) != NVFP4_OK)
         return NVFP4_ERR_CUDA;
-    g_launches++;
     if (rows > 0 && cols > 0) {
         nvfp4::SegRows seg;
         nvfp4_segment one = {0, rows};
         check_segments(&one, 1, rows, &seg);
-        const int grid = static_cast<int>(std::min<int64_t>(cdiv(rows, 8), int64_t(d->sm_count) * 8));
-        nvfp4::amax_kernel<<<grid, 256, 0, s>>>(static_cast<const uint16_t *>(X), rows, cols, ldx, seg, amax,
-                                                d->status);
+        const int64_t slices = amax_slices(rows, cols);
+        const int grid = static_cast<int>(std::min<int64_t>(cdiv(rows * slices, 8), int64_t(d->sm_count) * 8));
+        launch(nvfp4::amax_kernel, dim3(grid), dim3(256), 0, s, static_cast<const uint16_t *>(X), rows, cols, ldx, slices,
+               seg, amax, d->status);
         g_launches++;
         if (launch_ok() != NVFP4_OK)
             return NVFP4_ERR_CUDA;
     }
-    nvfp4::kv::kv_scale_kernel<<<1, 32, 0, s>>>(amax, scale);
+    launch(nvfp4::kv::kv_scale_kernel, dim3(1), dim3(32), 0, s, amax, scale);
     g_launches++;
     return launch_ok();
 }
@@ -992,7 +1034,7 @@ extern "C" int nvfp4_fp8_kv_quantize(const void *X, int64_t rows, int64_t cols, 
     p.status = d->status;
     const int64_t groups = rows * (cols / 8);
     const int grid = static_cast<int>(std::min<int64_t>(cdiv(groups, 256), int64_t(d->sm_count) * 16));
-    nvfp4::kv::kv_quantize_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(p);
+    launch(nvfp4::kv::kv_quantize_kernel, dim3(grid), dim3(256), 0, static_cast<cudaStream_t>(stream), p);
     g_launches++;
     return launch_ok();
 }

@@ -462,4 +462,20 @@ __device__ __forceinline__ uint32_t f32x2_to_e2m1x2(float lo, float hi)
     return out;
 }
 
+// ------------------------------------------- programmatic dependent launch
+// Every kernel of the library is launched so that the next kernel on the
+// stream may be scheduled before it finishes.  A kernel calls grid_dep_wait()
+// before its first access to global memory: it returns once the grids this
+// one depends on have completed and their writes are visible.  Right after
+// that it calls grid_dep_launch_dependents(), letting the next kernel's CTAs
+// start their own set-up; since that happens only after this grid's wait
+// returned, everything before this grid on the stream has completed by then.
+// Both are no-ops for a kernel launched without the attribute.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+__device__ __forceinline__ void grid_dep_launch_dependents()
+{
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 }  // namespace nvfp4

@@ -73,12 +73,28 @@ __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w 
 
 // ------------------------------------------------------------------ amax
 
+// words[0, n) = 0: clears amax accumulators in stream order as a kernel (so
+// the launches around it keep their programmatic dependencies).
+__global__ void zero_words_kernel(uint32_t *__restrict__ words, int32_t n)
+{
+    grid_dep_wait();
+    grid_dep_launch_dependents();
+    for (int i = threadIdx.x; i < n; i += blockDim.x)
+        words[i] = 0;
+}
+
 // amax_bits[seg] = max over the segment's rows of the bf16 magnitude bits
 // (the float max|x| is amax_bits << 16).  amax_bits must be zero on entry.
+// Each row is cut into `slices` contiguous ranges of 16-byte chunks, one warp
+// per (row, range): one range per row when there are rows enough to fill the
+// GPU, several when there are few (decode-sized inputs), so that a short
+// input is read by many warps at once instead of a few long loops.
 __global__ void __launch_bounds__(256) amax_kernel(const uint16_t *__restrict__ X, int64_t rows, int64_t K,
-                                                   int64_t ld, SegRows seg, uint32_t *__restrict__ amax_bits,
-                                                   uint32_t *__restrict__ status)
+                                                   int64_t ld, int64_t slices, SegRows seg,
+                                                   uint32_t *__restrict__ amax_bits, uint32_t *__restrict__ status)
 {
+    grid_dep_wait();
+    grid_dep_launch_dependents();
     __shared__ uint32_t s_max[kMaxSeg];
     if (threadIdx.x < kMaxSeg)
         s_max[threadIdx.x] = 0;
@@ -88,10 +104,14 @@ __global__ void __launch_bounds__(256) amax_kernel(const uint16_t *__restrict__ 
     const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
     const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
     const int64_t chunks = K >> 3;  // 16-byte chunks per row
+    const int64_t per_slice = (chunks + slices - 1) / slices;
 
     int slot = 0;
     uint32_t m = 0;
-    for (int64_t r = warp; r < rows; r += nwarps) {
+    for (int64_t item = warp; item < rows * slices; item += nwarps) {
+        const int64_t r = item / slices;
+        const int64_t c0 = (item - r * slices) * per_slice;
+        const int64_t c1 = min(c0 + per_slice, chunks);
         const int s = seg_of(seg, r);
         if (s != slot) {  // warp-uniform: every lane works on row r
             atomicMax(&s_max[slot], hmax16(m));
@@ -99,15 +119,15 @@ __global__ void __launch_bounds__(256) amax_kernel(const uint16_t *__restrict__ 
             slot = s;
         }
         const uint4 *p = reinterpret_cast<const uint4 *>(X + r * ld);
-        int64_t j = lane;
-        for (; j + 96 < chunks; j += 128) {
+        int64_t j = c0 + lane;
+        for (; j + 96 < c1; j += 128) {
             const uint4 a = __ldg(p + j), b = __ldg(p + j + 32), c = __ldg(p + j + 64), d = __ldg(p + j + 96);
             m = vmax_mag(m, a);
             m = vmax_mag(m, b);
             m = vmax_mag(m, c);
             m = vmax_mag(m, d);
         }
-        for (; j < chunks; j += 32)
+        for (; j < c1; j += 32)
             m = vmax_mag(m, __ldg(p + j));
     }
     atomicMax(&s_max[slot], hmax16(m));
@@ -211,6 +231,8 @@ __device__ __forceinline__ uint32_t quantize_block(const uint4 &v0, const uint4 
 // only write zero scale bytes.
 __global__ void __launch_bounds__(256) quantize_kernel(const QuantParams p)
 {
+    grid_dep_wait();
+    grid_dep_launch_dependents();
     __shared__ float s_g[kMaxSeg], s_rg[kMaxSeg];
     __shared__ int s_gok[kMaxSeg];
     if (threadIdx.x < p.seg.nseg) {
@@ -290,6 +312,8 @@ __global__ void __launch_bounds__(256) swiglu_kernel(const uint16_t *__restrict_
                                                      int32_t F, uint16_t *__restrict__ H,
                                                      uint32_t *__restrict__ amax_bits)
 {
+    grid_dep_wait();
+    grid_dep_launch_dependents();
     const uint32_t cpr = static_cast<uint32_t>(F) >> 3;
     const uint32_t total = static_cast<uint32_t>(rows) * cpr;
     uint32_t m = 0;
