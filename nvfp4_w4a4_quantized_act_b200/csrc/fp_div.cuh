@@ -41,4 +41,28 @@ __device__ __forceinline__ float div_shared(float x, float d, float r)
     return __fmaf_rn(-en, r, q);
 }
 
+// div_shared on the two bf16 values packed in w (low half first), with the
+// packed two-lane fp32 instructions of sm_100 (mul/fma .rn.f32x2): one
+// instruction per step for both quotients.  nr = -RN(1/d).  The steps run on
+// the negated dividends -x and the negated reciprocal, which gives the same
+// products, remainders and sums as div_shared (every negation is exact and
+// each fused operation sees the same operand values and signs), so the
+// results are bit-identical to it, signed zeros included.
+__device__ __forceinline__ void div_shared_x2(uint32_t w, float d, float nr, float &y_lo, float &y_hi)
+{
+    const uint32_t wn = w ^ 0x80008000u;  // -x, both halves
+    const float nx_lo = __uint_as_float(wn << 16);
+    const float nx_hi = __uint_as_float(wn & 0xFFFF0000u);
+    asm("{\n\t.reg .b64 x, q, e, dd, rr;\n\t"
+        "mov.b64 x, {%2, %3};\n\t"
+        "mov.b64 dd, {%4, %4};\n\t"
+        "mov.b64 rr, {%5, %5};\n\t"
+        "mul.rn.f32x2 q, x, rr;\n\t"      // q = (-x)(-r) = RN(x r)
+        "fma.rn.f32x2 e, dd, q, x;\n\t"   // e = RN(d q - x)
+        "fma.rn.f32x2 q, e, rr, q;\n\t"   // y = RN(q - e r)
+        "mov.b64 {%0, %1}, q;\n\t}"
+        : "=f"(y_lo), "=f"(y_hi)
+        : "f"(nx_lo), "f"(nx_hi), "f"(d), "f"(nr));
+}
+
 }  // namespace nvfp4

@@ -462,6 +462,22 @@ __device__ __forceinline__ uint32_t f32x2_to_e2m1x2(float lo, float hi)
     return out;
 }
 
+// Eight E2M1 codes (round to nearest even, saturating at +-6) packed into one
+// word: y[2i] in the low nibble and y[2i+1] in the high nibble of byte i.
+__device__ __forceinline__ uint32_t e2m1x8(const float (&y)[8])
+{
+    uint32_t out;
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+        "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+        : "=r"(out)
+        : "f"(y[0]), "f"(y[1]), "f"(y[2]), "f"(y[3]), "f"(y[4]), "f"(y[5]), "f"(y[6]), "f"(y[7]));
+    return out;
+}
+
 // ------------------------------------------- programmatic dependent launch
 // Every kernel of the library is launched so that the next kernel on the
 // stream may be scheduled before it finishes.  A kernel calls grid_dep_wait()

@@ -1,5 +1,6 @@
-// Compares the quantizer's shared-divisor division (div_shared, from
-// fp_div.cuh) with CUDA's IEEE division __fdiv_rn, bit for bit:
+// Compares the quantizer's shared-divisor division (div_shared and its packed
+// two-lane form div_shared_x2, from fp_div.cuh) with CUDA's IEEE division
+// __fdiv_rn, bit for bit (div_shared_x2 on the pair (x, -x)):
 //  (1) every bf16 significand x (128) against every fp32 significand d (2^23),
 //      with exponents chosen so x/d spans [2^-5, 2^5), both signs;
 //  (2) every finite bf16 value against pseudo-random divisors over the whole
@@ -13,6 +14,14 @@
 
 using nvfp4::div_shared;
 using nvfp4::div_shared_ok;
+using nvfp4::div_shared_x2;
+
+// bf16 bits of x (x is a bf16 value) in the low half, of -x in the high half
+__device__ uint32_t pair_of(float x)
+{
+    const uint32_t b = __float_as_uint(x) >> 16;
+    return b | ((b ^ 0x8000u) << 16);
+}
 
 __device__ unsigned int g_nrec;
 __device__ float g_rec[64][4];
@@ -53,6 +62,15 @@ __global__ void sweep_significands(unsigned long long *checked, unsigned long lo
                             record(xs, d, y, ref);
                         }
                         ++c;
+                        float y2lo, y2hi;
+                        div_shared_x2(pair_of(xs), d, -r, y2lo, y2hi);
+                        const float ref_neg = __fdiv_rn(-xs, d);
+                        if (__float_as_uint(y2lo) != __float_as_uint(ref) ||
+                            __float_as_uint(y2hi) != __float_as_uint(ref_neg)) {
+                            ++b;
+                            record(xs, d, y2lo, ref);
+                        }
+                        c += 2;
                     }
                 }
             }
@@ -83,18 +101,23 @@ __global__ void sweep_range(unsigned long long *checked, unsigned long long *bad
         if (!div_shared_ok(d, fabsf(x)))
             continue;
         ++a;
-        const float y = div_shared(x, d, __frcp_rn(d));
-        const float ref = __fdiv_rn(x, d);
+        const float r = __frcp_rn(d);
+        float y2[2];
+        div_shared_x2(pair_of(x), d, -r, y2[0], y2[1]);
+        const float ys[3] = {div_shared(x, d, r), y2[0], y2[1]};
+        const float refs[3] = {__fdiv_rn(x, d), __fdiv_rn(x, d), __fdiv_rn(-x, d)};
         // quotients >= 2^-20 must be the IEEE ones; smaller ones must stay below
         // 0.25 (all encode to +-0) with the sign of x
-        if (fabsf(ref) >= 0x1p-20f || fabsf(y) >= 0x1p-20f) {
-            if (__float_as_uint(y) != __float_as_uint(ref)) {
-                ++b;
-                record(x, d, y, ref);
+        for (int k = 0; k < 3; ++k) {
+            const float y = ys[k], ref = refs[k];
+            if (fabsf(ref) >= 0x1p-20f || fabsf(y) >= 0x1p-20f) {
+                if (__float_as_uint(y) != __float_as_uint(ref)) {
+                    ++b;
+                    record(x, d, y, ref);
+                }
+            } else {
+                b += (signbit(y) != signbit(ref)) || !(fabsf(y) < 0.25f);
             }
-            ++c;
-        } else {
-            b += (signbit(y) != signbit(ref)) || !(fabsf(y) < 0.25f);
             ++c;
         }
     }

@@ -1,7 +1,8 @@
 """The quantizer divides each block's 16 elements by one decode scale with a
-reciprocal plus one Markstein correction step (csrc/fp_div.cuh).  This test
-compiles a small CUDA program against that header and compares it, bit for
-bit, with CUDA's IEEE division __fdiv_rn: every bf16 significand against every
+reciprocal plus one Markstein correction step (csrc/fp_div.cuh), two
+quotients at a time with the packed f32x2 instructions.  This test compiles a
+small CUDA program against that header and compares both forms, bit for bit,
+with CUDA's IEEE division __fdiv_rn: every bf16 significand against every
 fp32 significand (both signs, quotients across ten binades), and every finite
 bf16 value against random divisors over the whole accepted range (quotients
 below 2^-20, which all encode to +-0, need only stay below 0.25 with the right
