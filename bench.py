@@ -341,6 +341,7 @@ def bench_gpu(args, rank, world, local):
     # quantize kernel throughput: one activation [8192, 5120] at HBM roofline
     quant = quantize_roofline(stack, pk, pk_kind)
     kv = fp8_kv_roofline(pk, pk_kind)
+    decode = decode_roofline(stack, pk, pk_kind)
 
     e2e = None
     if not args.no_e2e:
@@ -384,6 +385,7 @@ def bench_gpu(args, rank, world, local):
         },
         "quantize_roofline": quant,
         "fp8_kv_roofline": kv,
+        "decode_roofline": decode,
         "gemm_share_of_step": round(sum(gemm_ms) / ms_per_step, 4),
         "gpu_launches": int(launches),
         "clocks": clk,
@@ -469,6 +471,73 @@ def fp8_kv_roofline(pk, pk_kind):
             "algorithmic_bytes": int(alg), "peak_basis": pk_kind, "l2": "256 MB flush before each launch",
             "one_layer_k_cache_us": round(ms_layer * 1e3, 2),
             "one_layer_k_cache_gbs": round(TOKENS * 1024 * 3 / (ms_layer * 1e-3) / 1e9, 1)}
+
+
+def decode_roofline(stack, pk, pk_kind, token_counts=(1, 16, 64, 128)):
+    """Decode steps through the same 64-layer stack: M new tokens per step
+    (M <= 128 runs the split-K GEMM), every linear through the public calls
+    (nvfp4_linear_fused; nvfp4_linear_swiglu for gate/up; the down projection
+    re-quantizes h through nvfp4_linear_fused).  A step streams every NVFP4
+    weight once (13.4 GB, far above L2), so it is bound by HBM: the figure is
+    weight bytes per step / step time.  Each step is one CUDA graph of 256
+    linears (captured once per M, replayed)."""
+    from nvfp4_w4a4_quantized_act_b200 import ops
+    dev = stack.X.device
+    wbytes = sum(qw.codes.numel() + qw.sf.numel() for qs in stack.weights for qw in qs)
+    res = {"kernel": "split-K linear chain (amax + quantize + gemm_nvf4_kernel split-K + split sum) per linear",
+           "bound": "hbm", "unit": "GB/s", "peak": pk["hbm_gbs"], "peak_basis": pk_kind,
+           "weight_bytes_per_step": int(wbytes), "linears_per_step": 256, "steps": {}}
+    for M in token_counts:
+        X, X2, Y = stack.X[:M], stack.X2[:M], stack.Y[:M]
+        ws_bytes = max(ops.workspace_bytes(M, lin.N, lin.K, len(lin.segments))
+                       for _, lins in stack.layers for lin in lins)
+        ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+        h = torch.empty((M, 17408), dtype=torch.bfloat16, device=dev)
+        hc = torch.empty(M * 17408 // 2, dtype=torch.uint8, device=dev)
+        hsf = torch.empty(ops.sf_bytes(M, 17408), dtype=torch.uint8, device=dev)
+        gh = torch.empty(1, dtype=torch.float32, device=dev)
+        outs = {n: torch.empty((M, n), dtype=torch.bfloat16, device=dev) for n in (5120, 14432, 14336)}
+
+        def step():
+            for qs, (_, lins) in zip(stack.weights, stack.layers):
+                for lin, qw in zip(lins, qs):
+                    if lin.name == "gate_up":
+                        ops.linear_swiglu(X2, qw, h=h, h_codes=hc, h_sf=hsf, g_h=gh, ws=ws)
+                    elif lin.name == "down":
+                        ops.linear_fused(h, qw, out=outs[5120], ws=ws)
+                    else:
+                        src = Y if lin.name in ("gdn_out", "attn_o") else X
+                        if lin.N not in outs:
+                            outs[lin.N] = torch.empty((M, lin.N), dtype=torch.bfloat16, device=dev)
+                        ops.linear_fused(src, qw, out=outs[lin.N], ws=ws)
+
+        step()
+        torch.cuda.synchronize()
+        if ops.get_status() != 0:
+            raise RuntimeError("device status set by the decode step")
+        side = torch.cuda.Stream()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=side):
+            step()
+        for _ in range(3):
+            graph.replay()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(5):
+            s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s.record()
+            graph.replay()
+            e.record()
+            e.synchronize()
+            ts.append(s.elapsed_time(e))
+        del graph
+        if ops.get_status() != 0:
+            raise RuntimeError("device status set by the decode step")
+        ms = statistics.median(ts)
+        gbs = wbytes / (ms * 1e-3) / 1e9
+        res["steps"][str(M)] = {"us_per_step": round(ms * 1e3, 1), "us_per_linear": round(ms * 1e3 / 256, 2),
+                                "achieved": round(gbs, 1), "frac": round(gbs / pk["hbm_gbs"], 4)}
+    return res
 
 
 def bench_e2e(stack, args, world):

@@ -79,10 +79,13 @@ struct Params {
     // Split-K (single-CTA kernel, small M): work item t covers tile
     // t % num_tiles over the K steps of split t / num_tiles; with splits > 1
     // the epilogue writes alpha * acc as fp32 to partial[split][M][N] and a
-    // finalize kernel sums the splits in order.
+    // finalize kernel adds the splits in order.
     int32_t splits;
     int32_t kt_per_split;
     float *partial;
+    // the weight producer may load before the previous kernel on the stream
+    // has finished (that kernel does not write W)
+    int32_t w_early;
     int32_t kb_total;    // K / 64
     int32_t kt_total;    // ceil(kb_total / 4)
     int32_t n_row_tiles; // ceil(N / 128): scale tiles of W per K-step
@@ -339,9 +342,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     tc_fence_after();
     const uint32_t tmem = sm->tmem_base;
     // set-up above touches no global memory; from here on the previous
-    // kernel's outputs (the quantized activation) are read
-    grid_dep_wait();
-    grid_dep_launch_dependents();
+    // kernel's outputs (the quantized activation) are read.  With w_early the
+    // weight producer skips the wait: the kernel before this one does not
+    // write W, and everything before that kernel had completed when it
+    // allowed this launch, so the weights stream in while it finishes.
+    if (!(p.w_early && warp == 3)) {
+        grid_dep_wait();
+        grid_dep_launch_dependents();
+    }
 
     if (warp == 0 || warp == 3) {
         // ----------------------------------------------------- producers

@@ -290,6 +290,12 @@ int make_out_map(CUtensorMap *map, void *out, int64_t rows, int64_t cols)
 // K steps are divided into `splits` contiguous ranges that run as separate
 // work items.  The count depends on the shape alone (sized for 148 SMs), so
 // the result's bits do not depend on the device; every range is non-empty.
+//
+// The count minimises a cost model fitted to measurements on B200 at M <= 128:
+// a CTA spends about 0.6 us per K stage (its pipeline is latency-bound at
+// these sizes), while each split adds its fp32 partials (M x N x 4 bytes,
+// written with per-row stores and read back, about 1.5 TB/s together) and a
+// fixed cost for the finalize kernel that adds them (about 2 us).
 constexpr int kSplitKMax = 8;
 constexpr int kSplitKSms = 148;
 
@@ -300,9 +306,20 @@ int splitk_count(int64_t M, int64_t N, int64_t K)
         return 1;
     const int64_t tiles = cdiv(N, BN);
     const int64_t kt_total = cdiv(K / 64, KB_PER_STAGE);
-    const int64_t want = std::min<int64_t>({kSplitKMax, kt_total, std::max<int64_t>(1, kSplitKSms / tiles)});
-    const int64_t kps = cdiv(kt_total, want);
-    return static_cast<int>(cdiv(kt_total, kps));
+    const int64_t s_max = std::min<int64_t>({kSplitKMax, kt_total, std::max<int64_t>(1, kSplitKSms / tiles)});
+    int64_t best = 1;
+    double best_ns = 600.0 * static_cast<double>(kt_total);
+    for (int64_t want = 2; want <= s_max; ++want) {
+        const int64_t kps = cdiv(kt_total, want);
+        const int64_t S = cdiv(kt_total, kps);
+        const double ns = 600.0 * static_cast<double>(kps) +
+                          static_cast<double>(S * M * N) * 8.0 / 1500.0 + 2000.0;
+        if (ns < best_ns) {
+            best_ns = ns;
+            best = S;
+        }
+    }
+    return static_cast<int>(best);
 }
 
 // h_amax != nullptr selects the gated MLP epilogue (W is [gate | up]
@@ -312,7 +329,8 @@ int splitk_count(int64_t M, int64_t N, int64_t K)
 // second kernel.
 int run_gemm(DeviceState *d, const uint8_t *a_codes, const uint8_t *a_sf, const float *g_a, int64_t M, int64_t K,
              const uint8_t *w_codes, const uint8_t *w_sf, int64_t N, const nvfp4::SegRows &seg, const float *g_w,
-             void *out, unsigned flags, cudaStream_t stream, uint32_t *h_amax = nullptr, float *partial = nullptr)
+             void *out, unsigned flags, cudaStream_t stream, uint32_t *h_amax = nullptr, float *partial = nullptr,
+             bool w_early = false)
 {
     using namespace nvfp4::gemm;
     if (M == 0 || N == 0)
@@ -355,6 +373,7 @@ int run_gemm(DeviceState *d, const uint8_t *a_codes, const uint8_t *a_sf, const 
             p.partial = partial;
         }
     }
+    p.w_early = (w_early && !use_pair) ? 1 : 0;
     p.n_row_tiles = static_cast<int32_t>(n_row_tiles);
     p.sf_box_bytes = sf_box;
     p.sfb_box_rows = sfb_rows;
@@ -626,12 +645,13 @@ int nvfp4_linear_fused(const void *X, int64_t M, int64_t K, const uint8_t *w_cod
     check_segments(&one, 1, M, &one_seg);
     const bool dynamic = (flags & NVFP4_STATIC_SCALE) == 0;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    float *partial =
+        linear_partial_bytes(M, N, K) > 0 ? reinterpret_cast<float *>(base + linear_partial_off(M, K)) : nullptr;
     rc = run_quantize(d, X, M, K, K, one_seg, a_codes, a_sf, g_a, g_a, dynamic, amax, s);
     if (rc != NVFP4_OK)
         return rc;
-    float *partial =
-        linear_partial_bytes(M, N, K) > 0 ? reinterpret_cast<float *>(base + linear_partial_off(M, K)) : nullptr;
-    return run_gemm(d, a_codes, a_sf, g_a, M, K, w_codes, w_sf, N, seg, g_w, out, flags, s, nullptr, partial);
+    // the GEMM follows this call's own quantize kernel, which does not write W
+    return run_gemm(d, a_codes, a_sf, g_a, M, K, w_codes, w_sf, N, seg, g_w, out, flags, s, nullptr, partial, true);
 }
 
 int nvfp4_linear(const void *X, int64_t M, int64_t K, const uint8_t *w_codes, const uint8_t *w_sf, const float *g_w,
@@ -833,7 +853,8 @@ extern "C" int nvfp4_linear_fused_noalloc(const void *X, int64_t M, int64_t K, c
     rc = run_quantize(d, X, M, K, K, one_seg, a_codes, a_sf, g_a, g_a, true, amax, s);
     if (rc != NVFP4_OK)
         return rc;
-    return run_gemm(d, a_codes, a_sf, g_a, M, K, w_codes, w_sf, N, seg, g_w, out, flags, s);
+    // the GEMM follows this call's own quantize kernel, which does not write W
+    return run_gemm(d, a_codes, a_sf, g_a, M, K, w_codes, w_sf, N, seg, g_w, out, flags, s, nullptr, nullptr, true);
 }
 
 // ------------------------------------------------------ gated MLP (SwiGLU)
@@ -894,7 +915,8 @@ extern "C" int nvfp4_gemm_prequant_swiglu(const uint8_t *a_codes, const uint8_t 
     nvfp4::SegRows gu;
     const nvfp4_segment two[2] = {{0, F}, {F, 2 * F}};
     check_segments(two, 2, 2 * F, &gu);
-    return run_gemm(d, a_codes, a_sf, g_a, M, K, w_codes, w_sf, 2 * F, gu, g_w, h, 0, s, h_amax);
+    // the GEMM follows this call's own clearing of h_amax, which does not write W
+    return run_gemm(d, a_codes, a_sf, g_a, M, K, w_codes, w_sf, 2 * F, gu, g_w, h, 0, s, h_amax, nullptr, true);
 }
 
 extern "C" int nvfp4_linear_swiglu(const void *X, int64_t M, int64_t K, const uint8_t *w_codes, const uint8_t *w_sf,
@@ -944,7 +966,8 @@ extern "C" int nvfp4_linear_swiglu(const void *X, int64_t M, int64_t K, const ui
     nvfp4::SegRows gu;
     const nvfp4_segment two[2] = {{0, F}, {F, 2 * F}};
     check_segments(two, 2, 2 * F, &gu);
-    rc = run_gemm(d, a_codes, a_sf, g_a, M, K, w_codes, w_sf, 2 * F, gu, g_w, h, flags & NVFP4_SINGLE_CTA, s, h_amax);
+    rc = run_gemm(d, a_codes, a_sf, g_a, M, K, w_codes, w_sf, 2 * F, gu, g_w, h, flags & NVFP4_SINGLE_CTA, s, h_amax,
+                  nullptr, true);
     if (rc != NVFP4_OK)
         return rc;
     // h -> NVFP4 with the dynamic scale folded in by the epilogue

@@ -206,12 +206,14 @@ __device__ __forceinline__ uint32_t quantize_block(const uint4 &v0, const uint4 
             packed[i >> 2] |= ((lo << 3) | (hi << 7)) << ((i & 3) * 8);
         }
     } else if (div_shared_ok(d, bamax)) {
-        const float r = __frcp_rn(d);
+        const float nr = -__frcp_rn(d);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const float y0 = div_shared(bf16_lo(w[i]), d, r);
-            const float y1 = div_shared(bf16_hi(w[i]), d, r);
-            packed[i >> 2] |= f32x2_to_e2m1x2(y0, y1) << ((i & 3) * 8);
+        for (int h = 0; h < 2; ++h) {
+            float y[8];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                div_shared_x2(w[4 * h + i], d, nr, y[2 * i], y[2 * i + 1]);
+            packed[h] = e2m1x8(y);
         }
     } else {
 #pragma unroll

@@ -51,11 +51,17 @@ def _act_bytes(M, K):
     return sf_off + ops.sf_bytes(M, K)
 
 
+# split counts of the cost model in nvfp4_api.cu (0.6 us per K stage of a CTA
+# against the partials' bytes and the cost of their sum), worked by hand
 @pytest.mark.parametrize("M,N,K,splits", [
-    (16, 5120, 5120, 7),     # 20 tiles of 256 columns, 20 stages: 7 splits of <= 3 stages
-    (1, 1024, 5120, 7),      # 4 tiles: at most 8 splits, 20 stages -> 7 of <= 3
-    (128, 1280, 17408, 8),   # 68 stages: 8 splits of <= 9
-    (64, 16480, 5120, 2),    # 65 tiles: 148 // 65 = 2
+    (16, 5120, 5120, 5),     # 20 tiles, 20 stages: 5 splits of 4 stages
+    (1, 1024, 5120, 7),      # 4 tiles: 7 splits of <= 3 stages (8 would leave 3 per split too)
+    (3, 1000, 5120, 7),      # ragged N
+    (128, 1280, 17408, 7),   # 68 stages: 7 splits of <= 10
+    (16, 16480, 5120, 2),    # 65 tiles: at most 148 // 65 = 2
+    (64, 16480, 5120, 1),    # the partials would cost more than the stages saved
+    (128, 5120, 5120, 1),
+    (64, 5120, 5120, 3),
     (128, 34816, 5120, 1),   # 136 tiles fill the GPU: no split
     (16, 5120, 256, 1),      # one stage of K: no split
     (129, 5120, 5120, 1),    # more than one 128-row block: CTA-pair GEMM, no split

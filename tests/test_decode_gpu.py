@@ -74,23 +74,24 @@ def test_decode_linear_matches_oracle(M, N, K, widths):
 
 
 def test_split_sum_is_its_own_launch():
-    """K = 5120 at N = 5120 splits (one extra launch sums the partials); K =
-    256 has one stage, so it cannot split."""
-    X = wl.activation_normal(16, 5120, 1)
+    """K = 5120 at N = 5120 splits K (one more launch adds the partials);
+    K = 256 has one stage and cannot split."""
     W, _ = _weight(5120, 5120, None, 1)
     qw = ops.quantize_weights(W.to(DEV))
-    Xs = X[:, :256].contiguous()
     qs = ops.quantize_weights(W[:, :256].contiguous().to(DEV))
-    ops.linear(X.to(DEV), qw)
-    ops.linear(Xs.to(DEV), qs)
-    torch.cuda.synchronize()
-    n0 = ops.launch_count()
-    ops.linear(X.to(DEV), qw)
-    n1 = ops.launch_count()
-    ops.linear(Xs.to(DEV), qs)
-    n2 = ops.launch_count()
+
+    def launches(M, K, q):
+        X = wl.activation_normal(M, K, 1).to(DEV)
+        ops.linear(X, q)
+        torch.cuda.synchronize()
+        n0 = ops.launch_count()
+        ops.linear(X, q)
+        return ops.launch_count() - n0
+
+    unsplit = launches(16, 256, qs)
+    assert launches(1, 5120, qw) == unsplit + 1
+    assert launches(16, 5120, qw) == unsplit + 1
     assert ops.get_status() == 0
-    assert (n1 - n0) == (n2 - n1) + 1
 
 
 def test_zero_activation_and_single_row():

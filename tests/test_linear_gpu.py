@@ -84,8 +84,8 @@ def test_single_global_scale_mismatch_is_reproduced():
     bad = host(ops.linear_fused(X.to(DEV), bad_w, out_fp32=True))
     g = host(qw.g_w)
     assert len(set(g.tolist())) == len(segs)
-    # M = 128 splits K in two: each partial is scaled before the two are
-    # added, so the identity holds to an ulp of the partials' magnitude
+    # where K is split (small M) each partial is scaled before the partials
+    # are added, so the identity holds to an ulp of the partials' magnitude
     # (cancellation can make that many ulps of a small output)
     for (a, b), gm in zip(segs, g):
         ratio = np.float64(g[0]) / np.float64(gm)
