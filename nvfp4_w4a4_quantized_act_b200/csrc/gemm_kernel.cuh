@@ -402,6 +402,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             int stage = 0;
             uint32_t phase = 0;
             int local = 0;
+            // Operand descriptors of stage 0; a stage adds STAGE_BYTES and a
+            // K-step 32 bytes to the 14-bit start-address field (shared
+            // addresses stay below 2^18, so it never carries).  Computing them
+            // once keeps the gap between two stages' MMAs short.
+            const uint64_t adesc0 = smem_desc(a_smem(0), 16, 1024, 2);
+            const uint64_t bdesc0 = smem_desc(b_smem(0), 16, 1024, 2);
+            constexpr uint32_t HALF_B = (HALF_N * BK_BYTES) >> 4;  // second 128 rows of W
             for (int item = blockIdx.x; item < p.num_tiles * p.splits && !sm->abort_flag;
                  item += gridDim.x, ++local) {
                 int tile, split, kt0, kt1;
@@ -423,16 +430,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     const int nkb = min(KB_PER_STAGE, p.kb_total - kt * KB_PER_STAGE);
                     const uint32_t sfa_t = tmem + SF_COL0 + stage * SF_BUF_COLS;
                     const uint32_t sfb_t = sfa_t + 4 * KB_PER_STAGE;
+                    const uint32_t soff = (static_cast<uint32_t>(stage) * STAGE_BYTES) >> 4;
+                    const uint64_t ad = adesc0 + soff, bd = bdesc0 + soff;
                     for (int kb = 0; kb < nkb; ++kb) {
-                        const uint64_t adesc = smem_desc(a_smem(stage) + kb * 32, 16, 1024, 2);
                         const uint32_t acc_flag = (kt > kt0 || kb > 0) ? 1u : 0u;
 #pragma unroll
-                        for (int h = 0; h < 2; ++h) {
-                            const uint64_t bdesc =
-                                smem_desc(b_smem(stage) + h * (HALF_N * BK_BYTES) + kb * 32, 16, 1024, 2);
-                            tc_mma_nvf4(tmem + h * HALF_N, adesc, bdesc, IDESC, sfa_t + kb * 4,
-                                        sfb_t + kb * 8 + h * 4, acc_flag);
-                        }
+                        for (int h = 0; h < 2; ++h)
+                            tc_mma_nvf4(tmem + h * HALF_N, ad + 2 * kb, bd + h * HALF_B + 2 * kb, IDESC,
+                                        sfa_t + kb * 4, sfb_t + kb * 8 + h * 4, acc_flag);
                     }
                     tc_commit(smem_u32(&sm->empty[stage]));
                     if (++stage == STAGES) {

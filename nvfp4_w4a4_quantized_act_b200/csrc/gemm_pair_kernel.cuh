@@ -258,6 +258,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
             int stage = 0;
             uint32_t phase = 0;
             int local = 0;
+            // Operand descriptors of stage 0; a stage adds STAGE_BYTES and a
+            // K-step 32 bytes to the 14-bit start-address field (shared
+            // addresses stay below 2^18, so the field never carries).  Kept
+            // out of the gap between one stage's last MMA and the next
+            // stage's first, where the tensor pipe has at most one MMA queued.
+            const uint64_t adesc0 = smem_desc(a_smem(0), 16, 1024, 2);
+            const uint64_t bdesc0 = smem_desc(b_smem(0), 16, 1024, 2);
+            const uint32_t full0 = smem_u32(&sm->full[0]), empty0 = smem_u32(&sm->empty[0]);
+            const int kt_whole = p.kb_total / KB_PER_STAGE;  // stages with all four K-steps
             for (int tile = cid; tile < p.pair_tiles && !sm->abort_flag; tile += ncl, ++local) {
                 if (!mbar_wait_bounded_cluster(smem_u32(&sm->acc_empty), (local & 1) ^ 1u, p.wait_limit_ns)) {
                     raise_timeout_pair(sm, p.status);
@@ -266,22 +275,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                 tc_fence_after();
                 bool ok = true;
                 for (int kt = 0; kt < p.kt_total; ++kt) {
+                    const uint32_t soff = (static_cast<uint32_t>(stage) * STAGE_BYTES) >> 4;
+                    const uint64_t ad = adesc0 + soff, bd = bdesc0 + soff;
+                    const uint32_t sf_t = tmem + SF_COL0 + stage * SF_BUF_COLS;
+                    const uint32_t acc0 = kt > 0 ? 1u : 0u;
                     // codes of both CTAs landed and the stage's scales are in TMEM
-                    if (!mbar_wait_bounded(smem_u32(&sm->full[stage]), phase, p.wait_limit_ns)) {
+                    if (!mbar_wait_bounded(full0 + 8u * stage, phase, p.wait_limit_ns)) {
                         raise_timeout_pair(sm, p.status);
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const int nkb = min(KB_PER_STAGE, p.kb_total - kt * KB_PER_STAGE);
-                    const uint32_t sf_t = tmem + SF_COL0 + stage * SF_BUF_COLS;
-                    for (int kb = 0; kb < nkb; ++kb) {
-                        const uint64_t adesc = smem_desc(a_smem(stage) + kb * 32, 16, 1024, 2);
-                        const uint64_t bdesc = smem_desc(b_smem(stage) + kb * 32, 16, 1024, 2);
-                        tc_mma_pair_nvf4(tmem, adesc, bdesc, IDESC, sf_t + kb * 4, sf_t + 16 + kb * 8,
-                                         (kt > 0 || kb > 0) ? 1u : 0u);
+                    if (kt < kt_whole) {
+#pragma unroll
+                        for (int kb = 0; kb < KB_PER_STAGE; ++kb)
+                            tc_mma_pair_nvf4(tmem, ad + 2 * kb, bd + 2 * kb, IDESC, sf_t + kb * 4, sf_t + 16 + kb * 8,
+                                             kb > 0 ? 1u : acc0);
+                    } else {
+                        const int nkb = p.kb_total - kt * KB_PER_STAGE;
+                        for (int kb = 0; kb < nkb; ++kb)
+                            tc_mma_pair_nvf4(tmem, ad + 2 * kb, bd + 2 * kb, IDESC, sf_t + kb * 4, sf_t + 16 + kb * 8,
+                                             kb > 0 ? 1u : acc0);
                     }
-                    tc_commit_pair_both(smem_u32(&sm->empty[stage]), 3);
+                    tc_commit_pair_both(empty0 + 8u * stage, 3);
                     if (++stage == STAGES) {
                         stage = 0;
                         phase ^= 1u;
