@@ -50,7 +50,7 @@ FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1
 # one layer, from one ncu capture of this kernel source (profiles/
 # gemm_nvf4_pair_kernel_layer_8192tok.md gives the command).  Reported only
 # while the kernel sources still have the captured hash.
-GEMM_TRAFFIC = {"source_sha256_12": "aa7977a091bd", "bytes_per_launch": 329.310e6}
+GEMM_TRAFFIC = {"source_sha256_12": "78f8748fe9f7", "bytes_per_launch": 331.262e6}
 GEMM_SOURCES = [os.path.join(ROOT, "nvfp4_w4a4_quantized_act_b200", "csrc", f)
                 for f in ("gemm_kernel.cuh", "gemm_pair_kernel.cuh", "ptx_sm100.cuh")]
 
@@ -77,6 +77,8 @@ def parse_args():
     ap.add_argument("--layers", type=int, default=64, help="layers in the stack (64 = the full model)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-side", action="store_true",
+                    help="skip the side measurements (quantize, FP8 KV cache, decode) after the timed steps")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     return ap.parse_args()
 
@@ -339,9 +341,11 @@ def bench_gpu(args, rank, world, local):
     fp4_peak = pk["bf16_tflops_sustained"] * FP4_PER_BF16
 
     # quantize kernel throughput: one activation [8192, 5120] at HBM roofline
-    quant = quantize_roofline(stack, pk, pk_kind)
-    kv = fp8_kv_roofline(pk, pk_kind)
-    decode = decode_roofline(stack, pk, pk_kind)
+    quant = kv = decode = None
+    if not args.no_side:
+        quant = quantize_roofline(stack, pk, pk_kind)
+        kv = fp8_kv_roofline(pk, pk_kind)
+        decode = decode_roofline(stack, pk, pk_kind)
 
     e2e = None
     if not args.no_e2e:
