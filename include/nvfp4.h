@@ -31,6 +31,13 @@
  *    multiples of 8 elements (NVFP4_ERR_MISALIGNED otherwise).
  *  - Weights use the nn.Linear layout W[N, K]; a linear computes
  *    out[M, N] = X[M, K] * W^T.
+ *  - Kernels are launched with programmatic stream serialization: each one
+ *    waits (griddepcontrol.wait) for the work before it on the stream and
+ *    then lets the next kernel start its set-up early.  Stream order is kept
+ *    for every ordinary launch; a caller's own kernel launched after ours
+ *    with cudaLaunchAttributeProgrammaticStreamSerialization must call
+ *    cudaGridDependencySynchronize() before reading our outputs, as with any
+ *    such launch.  Calls can be captured in CUDA graphs.
  *
  * NVFP4 storage produced and consumed here:
  *  - codes: [rows, K/2] bytes, row-major; byte i of a row holds element 2i in
