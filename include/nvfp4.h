@@ -274,7 +274,7 @@ uint64_t nvfp4_launch_count(void);
  * The first call on a device looks up the array's device address (once per
  * device, with that device current); make that first call before any stream
  * capture begins.  All calls share the one array and it keeps the last
- * call's contents (the amax word is cleared by every call): calls that can
+ * call's contents (no call reads what an earlier call left there): calls that can
  * overlap on the GPU -- on different streams without ordering, or from
  * several host threads -- race with each other and must be serialized by the
  * caller. */
@@ -288,8 +288,8 @@ int nvfp4_linear_fused_noalloc(const void *X, int64_t M, int64_t K,
 /* ------------------------------------------------- FP8 KV-cache (E4M3)
  *
  * The attention KV cache in FP8 E4M3 with one calibrated FP32 scale per cache
- * tensor: the pages' recipe is to "ship the calibrated KV-cache scales",
- * which they report as performance-free (freegardner.com, "Quantizing All
+ * tensor: the pages' recipe ships calibrated scales for the KV cache along
+ * with the weights and reports them as costing nothing (freegardner.com, "Quantizing All
  * Layers Reveals Recurrent Memory Is Robust", section "The Calibrated Cache
  * That Ships for Free"; thevalue.engineering, "NVFP4 W4A4 quantization
  * compresses 27B hybrid models", section "Efficiency Gains and Serving

@@ -5,7 +5,7 @@
 //   out[m, n] = round( acc[m, n] * fl32(g_a * g_w[seg(n)]) )
 //   acc[m, n] = sum_k qa[m,k] sa[m,k/16] qw[n,k] sw[n,k/16]   (fp32, TMEM)
 //
-// The block-scaled product runs "natively on current tensor cores" ("Why
+// The block-scaled product runs on the tensor cores without emulation ("Why
 // Gated DeltaNet Survives 4-Bit Quantization", kipquest.com, "The deep
 // dive"); applying each module's own FP32 global scale to its columns is the
 // repair of the global-scale mismatch that appears when per-module-calibrated

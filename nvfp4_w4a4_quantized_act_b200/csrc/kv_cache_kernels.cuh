@@ -1,6 +1,6 @@
 // kv_cache_kernels.cuh -- FP8 (E4M3) KV-cache quantization with a calibrated
-// per-tensor scale: "ship the calibrated KV-cache scales", which are
-// performance-free when calibrated (freegardner.com, "Quantizing All Layers
+// per-tensor scale: the recipe ships calibrated KV-cache scales, which the
+// pages report as costing nothing (freegardner.com, "Quantizing All Layers
 // Reveals Recurrent Memory Is Robust", section "The Calibrated Cache That
 // Ships for Free"; thevalue.engineering, "NVFP4 W4A4 quantization compresses
 // 27B hybrid models", section "Efficiency Gains and Serving Optimization").

@@ -3,8 +3,8 @@ weights through one fused GEMM with a single global scale does to each
 module's outputs, and what each repair leaves.
 
 The pages describe the fault: checkpoints calibrated per module, served by
-kernels that fuse those modules into one matrix multiply, come out wrong (it
-"silently corrupts the gates") -- kipquest.com, "Why Gated DeltaNet Survives
+kernels that fuse those modules into one matrix multiply, come out wrong (the
+gates are corrupted with no error raised) -- kipquest.com, "Why Gated DeltaNet Survives
 4-Bit Quantization", sections "The abstract" and "The deep dive".  They give
 no error figures; this measures them on synthetic tensors shaped like the GDN
 input projection (q, k, v, z, b, a: N = 16480 in six modules whose weight

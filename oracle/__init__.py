@@ -305,7 +305,7 @@ def silu_mul(g: np.ndarray, u: np.ndarray) -> np.ndarray:
 
 # ------------------------------------------------------ FP8 KV-cache codec
 # The KV cache in FP8 (E4M3) with one calibrated FP32 decode scale per cache
-# tensor ("ship the calibrated KV-cache scales": freegardner.com, section
+# tensor (the recipe ships calibrated KV-cache scales: freegardner.com, section
 # "The Calibrated Cache That Ships for Free"; thevalue.engineering, section
 # "Efficiency Gains and Serving Optimization").  Readings: s = amax / 448,
 # code = E4M3_RNE_satfinite(x / s), sign kept.
