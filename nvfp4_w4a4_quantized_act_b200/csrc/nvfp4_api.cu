@@ -165,12 +165,6 @@ int64_t amax_slices(int64_t rows, int64_t cols)
     return std::max<int64_t>(1, cdiv(cols >> 3, 128));
 }
 
-// Dynamic-scale tensors up to this many bytes (one segment) are quantized by
-// one cluster of CTAs in one launch (quantize_small_kernel); measured on
-// B200, the clear + amax + quantize launches cost ~4.3 us however small the
-// tensor.
-constexpr int64_t kSmallQuantBytes = 160 * 1024;
-
 int run_quantize(DeviceState *d, const void *X, int64_t rows, int64_t K, int64_t ld, const nvfp4::SegRows &seg,
                  uint8_t *codes, uint8_t *sf, const float *g_in, float *g_out, bool dynamic, uint32_t *amax_ws,
                  cudaStream_t stream, int64_t gate_up_F = 0)
@@ -179,9 +173,7 @@ int run_quantize(DeviceState *d, const void *X, int64_t rows, int64_t K, int64_t
     const int64_t groups = cdiv(K, 64);
     if (rows_pad * groups * 4 >= (int64_t(1) << 31) || K > (int64_t(1) << 30))
         return NVFP4_ERR_UNSUPPORTED_SHAPE;
-    // a small single-segment tensor (decode-sized) takes one launch
-    const bool small = dynamic && seg.nseg == 1 && gate_up_F == 0 && rows * K * 2 <= kSmallQuantBytes;
-    if (dynamic && !small) {
+    if (dynamic) {
         if (zero_words(amax_ws, seg.nseg, stream) != NVFP4_OK)
             return NVFP4_ERR_CUDA;
         if (rows > 0) {
@@ -210,11 +202,6 @@ int run_quantize(DeviceState *d, const void *X, int64_t rows, int64_t K, int64_t
     p.codes = codes;
     p.sf = sf;
     p.gate_up_F = static_cast<int32_t>(gate_up_F);
-    if (small) {
-        launch(nvfp4::quantize_small_kernel, dim3(nvfp4::SMALL_QUANT_CTAS), dim3(1024), 0, stream, p, d->status);
-        g_launches++;
-        return launch_ok();
-    }
     const int64_t threads = rows_pad * groups * 4;
     int grid = static_cast<int>(std::min<int64_t>(std::max<int64_t>(cdiv(threads, 256), 1), int64_t(d->sm_count) * 16));
     launch(nvfp4::quantize_kernel, dim3(grid), dim3(256), 0, stream, p);

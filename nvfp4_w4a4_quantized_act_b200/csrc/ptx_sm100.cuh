@@ -325,14 +325,6 @@ __device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr)
 }
 
 // Every thread of every CTA of the cluster arrives, then waits for all.
-// 32-bit load from shared memory of a CTA of this cluster (address from mapa).
-__device__ __forceinline__ uint32_t ld_shared_cluster_u32(uint32_t addr)
-{
-    uint32_t v;
-    asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
-    return v;
-}
-
 __device__ __forceinline__ void cluster_sync_all()
 {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");

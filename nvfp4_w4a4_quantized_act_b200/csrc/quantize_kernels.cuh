@@ -231,16 +231,27 @@ __device__ __forceinline__ uint32_t quantize_block(const uint4 &v0, const uint4 
 // items; the next item's input is loaded before the current one is
 // quantized.  Rows past `rows` (up to the 128-row padding) and blocks past K
 // only write zero scale bytes.
-// The items of quantize_kernel handled by warps warp0, warp0 + nwarps, ...
-// with the per-segment scales already in s_g / s_rg / s_gok.
-// Rows [item_rows, rows_pad) are left to the caller.
-__device__ __forceinline__ void quantize_items(const QuantParams &p, const float *s_g, const float *s_rg,
-                                               const int *s_gok, uint32_t warp0, uint32_t nwarps,
-                                               uint32_t item_rows)
+__global__ void __launch_bounds__(256) quantize_kernel(const QuantParams p)
 {
+    grid_dep_wait();
+    grid_dep_launch_dependents();
+    __shared__ float s_g[kMaxSeg], s_rg[kMaxSeg];
+    __shared__ int s_gok[kMaxSeg];
+    if (threadIdx.x < p.seg.nseg) {
+        const float g = (p.mode == 0) ? global_scale_from_amax(p.amax_bits[threadIdx.x]) : p.g_in[threadIdx.x];
+        s_g[threadIdx.x] = g;
+        s_rg[threadIdx.x] = __frcp_rn(g);
+        s_gok[threadIdx.x] = (g >= 0x1p-80f && g <= 0x1p100f) ? 1 : 0;
+        if (p.mode == 0 && p.g_out != nullptr && blockIdx.x == 0)
+            p.g_out[threadIdx.x] = g;
+    }
+    __syncthreads();
+
     const int lane = threadIdx.x & 31;
     const uint32_t cpr = (static_cast<uint32_t>(p.groups) + 7u) >> 3;  // chunks per row
-    const uint32_t items = item_rows * cpr;
+    const uint32_t items = static_cast<uint32_t>(p.rows_pad) * cpr;
+    const uint32_t warp0 = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const uint32_t nwarps = (gridDim.x * blockDim.x) >> 5;
     const uint32_t drow = nwarps / cpr, dchunk = nwarps - drow * cpr;
     const int nblk = p.K >> 4;
     const bool one_seg = p.seg.nseg == 1;
@@ -291,88 +302,6 @@ __device__ __forceinline__ void quantize_items(const QuantParams &p, const float
         chunk = nchunk;
         v0 = n0;
         v1 = n1;
-    }
-}
-
-__global__ void __launch_bounds__(256) quantize_kernel(const QuantParams p)
-{
-    grid_dep_wait();
-    grid_dep_launch_dependents();
-    __shared__ float s_g[kMaxSeg], s_rg[kMaxSeg];
-    __shared__ int s_gok[kMaxSeg];
-    if (threadIdx.x < p.seg.nseg) {
-        const float g = (p.mode == 0) ? global_scale_from_amax(p.amax_bits[threadIdx.x]) : p.g_in[threadIdx.x];
-        s_g[threadIdx.x] = g;
-        s_rg[threadIdx.x] = __frcp_rn(g);
-        s_gok[threadIdx.x] = (g >= 0x1p-80f && g <= 0x1p100f) ? 1 : 0;
-        if (p.mode == 0 && p.g_out != nullptr && blockIdx.x == 0)
-            p.g_out[threadIdx.x] = g;
-    }
-    __syncthreads();
-    quantize_items(p, s_g, s_rg, s_gok, (blockIdx.x * blockDim.x + threadIdx.x) >> 5, (gridDim.x * blockDim.x) >> 5,
-                   static_cast<uint32_t>(p.rows_pad));
-}
-
-// Dynamic-scale quantization of a small tensor (one segment, decode-sized)
-// in one launch: a cluster of SMALL_QUANT_CTAS CTAs reduces max|X| (each CTA
-// in shared memory, then every CTA reads the others' maxima through
-// distributed shared memory between two cluster barriers), forms g =
-// amax/2688 and quantizes the rows with all the cluster's warps; the
-// padding rows of the last scale tile get their zero scale words directly.
-// Replaces the clear + amax + quantize launches.
-constexpr int SMALL_QUANT_CTAS = 8;
-
-__global__ void __cluster_dims__(SMALL_QUANT_CTAS, 1, 1) __launch_bounds__(1024)
-    quantize_small_kernel(const QuantParams p, uint32_t *__restrict__ status)
-{
-    grid_dep_wait();
-    grid_dep_launch_dependents();
-    __shared__ uint32_t s_max;
-    __shared__ float s_g[kMaxSeg], s_rg[kMaxSeg];
-    __shared__ int s_gok[kMaxSeg];
-    if (threadIdx.x == 0)
-        s_max = 0;
-    __syncthreads();
-    const uint32_t nthreads = SMALL_QUANT_CTAS * blockDim.x;
-    const uint32_t tid = blockIdx.x * blockDim.x + threadIdx.x;
-    // max|x| over [rows, K] (16-byte loads; K % 16 == 0, ld % 8 == 0)
-    const int64_t chunks = static_cast<int64_t>(p.K) >> 3;
-    const int64_t total = static_cast<int64_t>(p.rows) * chunks;
-    uint32_t m = 0;
-    for (int64_t i = tid; i < total; i += nthreads) {
-        const int64_t r = i / chunks, c = i - r * chunks;
-        m = vmax_mag(m, __ldg(reinterpret_cast<const uint4 *>(p.X + r * p.ld) + c));
-    }
-    uint32_t v = hmax16(m);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1)
-        v = max(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
-    if ((threadIdx.x & 31) == 0 && v != 0)
-        atomicMax(&s_max, v);
-    cluster_sync_all();  // every CTA's maximum is final (and visible in the cluster)
-    if (threadIdx.x == 0) {
-        uint32_t a = 0;
-        for (int r = 0; r < SMALL_QUANT_CTAS; ++r)
-            a = max(a, ld_shared_cluster_u32(mapa_shared(smem_u32(&s_max), r)));
-        if (a >= 0x7F80u && blockIdx.x == 0)  // Inf or NaN magnitude
-            atomicOr(status, kStatusNonFinite);
-        const float g = global_scale_from_amax(a);
-        s_g[0] = g;
-        s_rg[0] = __frcp_rn(g);
-        s_gok[0] = (g >= 0x1p-80f && g <= 0x1p100f) ? 1 : 0;
-        if (p.g_out != nullptr && blockIdx.x == 0)
-            p.g_out[0] = g;
-    }
-    cluster_sync_all();  // no CTA leaves while another still reads its s_max
-    quantize_items(p, s_g, s_rg, s_gok, tid >> 5, nthreads >> 5, static_cast<uint32_t>(p.rows));
-    // zero scale words of the padding rows [rows, rows_pad)
-    const uint32_t npad = static_cast<uint32_t>(p.rows_pad - p.rows) * static_cast<uint32_t>(p.groups);
-    for (uint32_t i = tid; i < npad; i += nthreads) {
-        const uint32_t r = static_cast<uint32_t>(p.rows) + i / static_cast<uint32_t>(p.groups);
-        const uint32_t cg = i % static_cast<uint32_t>(p.groups);
-        const uint64_t tile = static_cast<uint64_t>(r >> 7) * p.groups + cg;
-        const uint32_t rr = r & 127u;
-        *reinterpret_cast<uint32_t *>(p.sf + tile * 512 + (rr & 31u) * 16 + (rr >> 5) * 4) = 0u;
     }
 }
 
