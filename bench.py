@@ -456,7 +456,10 @@ def quantize_roofline(stack, pk, pk_kind):
             "l2": "256 MB written and read back before each launch",
             "static_scale_us": round(ms_static * 1e3, 2),
             "static_scale_gbs": round(alg / (ms_static * 1e-3) / 1e9, 1),
-            "torch_read_of_x_us": round(ms_read * 1e3, 2)}
+            "torch_read_of_x_us": round(ms_read * 1e3, 2),
+            "torch_read_of_x_gbs": round(X.numel() * 2 / (ms_read * 1e-3) / 1e9, 1),
+            # the calibrated single pass's byte rate against a plain read of X of the same size
+            "static_frac_of_plain_read_rate": round((alg / ms_static) / (X.numel() * 2 / ms_read), 3)}
 
 
 def fp8_kv_roofline(pk, pk_kind):
