@@ -48,9 +48,10 @@ FP4_PER_BF16 = 4.0  # dense FP4 : dense BF16 tensor throughput on B200 (9 : 2.25
 FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # DRAM bytes (read + write) per GEMM launch, mean over the four GEMM launches of
 # one layer, from one ncu capture of this kernel source (profiles/
-# gemm_nvf4_pair_kernel_layer_8192tok.md gives the command).  Reported only
+# gemm_nvf4_pair_kernel_layer_8192tok.md gives the command: the DRAM-bytes
+# capture).  Reported only
 # while the kernel sources still have the captured hash.
-GEMM_TRAFFIC = {"source_sha256_12": "78f8748fe9f7", "bytes_per_launch": 331.262e6}
+GEMM_TRAFFIC = {"source_sha256_12": "30d7b96c8d71", "bytes_per_launch": 333.045e6}
 GEMM_SOURCES = [os.path.join(ROOT, "nvfp4_w4a4_quantized_act_b200", "csrc", f)
                 for f in ("gemm_kernel.cuh", "gemm_pair_kernel.cuh", "ptx_sm100.cuh")]
 
