@@ -25,6 +25,7 @@ CASES = [
     (64, 16480, 5120, [2048, 2048, 6144, 6144, 48, 48]),
     (128, 1280, 17408, None),
     (100, 5120, 2048, [4096, 1024]),
+    (3, 1002, 5120, [500, 502]),  # N % 4 != 0: scalar partial and output stores
 ]
 
 
