@@ -162,7 +162,12 @@ int nvfp4_gemm_prequant(const uint8_t *a_codes, const uint8_t *a_sf, const float
  * split into nseg modules, each with its own global scale g_w[m].
  * X: bf16 [M, K] contiguous.  ws: nvfp4_workspace_bytes(M, N, K, nseg)
  * bytes.  With NVFP4_STATIC_SCALE the activation scale is read from the
- * first float of ws + 256 (see nvfp4_linear_act_scale_offset()). */
+ * first float of ws + 256 (see nvfp4_linear_act_scale_offset()).
+ * Decode-sized inputs (M <= 128) may divide K among several CTAs (split-K):
+ * each writes alpha * acc in fp32 to the workspace and a second kernel adds
+ * the splits in a fixed order, so results are deterministic and the same on
+ * every device, though their last bits can differ from nvfp4_gemm_prequant
+ * (which never splits) on the same operands; both meet the same tolerance. */
 int nvfp4_linear_fused(const void *X, int64_t M, int64_t K,
                        const uint8_t *w_codes, const uint8_t *w_sf, int64_t N,
                        const nvfp4_segment *segs, const float *g_w, int nseg,
