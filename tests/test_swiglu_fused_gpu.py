@@ -72,9 +72,10 @@ def _check(M, K, F, X, W, rows, cols, single_cta=False):
 
 
 @pytest.mark.parametrize("single_cta", [False, True])
-@pytest.mark.parametrize("M,K,F", [(200, 512, 384), (300, 768, 640)])
+@pytest.mark.parametrize("M,K,F", [(200, 512, 384), (300, 768, 640), (1, 512, 384), (77, 256, 256)])
 def test_linear_swiglu_small_full_check(M, K, F, single_cta):
-    """Every h value: M > 128 runs the CTA-pair kernel unless single_cta."""
+    """Every h value: M > 128 runs the CTA-pair kernel unless single_cta;
+    decode-sized M (one partial 128-row block) the single-CTA gated kernel."""
     X = wl.activation_normal(M, K, 51 + M)
     W = _gate_up(F, K, 52 + F)
     _check(M, K, F, X, W, np.arange(M), np.arange(F), single_cta)
