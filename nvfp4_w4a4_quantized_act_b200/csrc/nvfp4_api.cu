@@ -152,10 +152,6 @@ int zero_words(uint32_t *words, int n, cudaStream_t stream)
     return launch_ok();
 }
 
-// K1 + K2 for `rows` x K bf16 rows, segment table `seg`.  mode 0: dynamic
-// scale from max|x| (amax words in ws, g written to g_out); mode 1: scale
-// read from g_in.
-//
 // Rows of the amax pass are cut into ranges of 128 16-byte chunks (one
 // four-load sweep of a warp) while rows are too few to give every SM work.
 int64_t amax_slices(int64_t rows, int64_t cols)
@@ -165,6 +161,39 @@ int64_t amax_slices(int64_t rows, int64_t cols)
     return std::max<int64_t>(1, cdiv(cols >> 3, 128));
 }
 
+// max|x| per segment into amax_ws (bf16 magnitude bits).  A tensor of at
+// most 32 KB (decode-sized) is read by one CTA of 32 warps that stores the
+// result, so the words need no clearing launch first; larger ones are cleared
+// and reduced across the grid with atomics.
+constexpr int64_t kOneBlockAmaxBytes = 32 * 1024;
+
+int run_amax(DeviceState *d, const void *X, int64_t rows, int64_t K, int64_t ld, const nvfp4::SegRows &seg,
+             uint32_t *amax_ws, cudaStream_t stream)
+{
+    if (rows > 0 && rows * K * 2 <= kOneBlockAmaxBytes) {
+        const int64_t slices = std::max<int64_t>(amax_slices(rows, K), cdiv(32, rows));
+        launch(nvfp4::amax_kernel, dim3(1), dim3(1024), 0, stream, static_cast<const uint16_t *>(X), rows, K, ld,
+               slices, seg, amax_ws, d->status, static_cast<int32_t>(1));
+        g_launches++;
+        return launch_ok();
+    }
+    if (zero_words(amax_ws, seg.nseg, stream) != NVFP4_OK)
+        return NVFP4_ERR_CUDA;
+    if (rows > 0) {
+        const int64_t slices = amax_slices(rows, K);
+        const int64_t warps_needed = rows * slices;
+        const int grid = static_cast<int>(std::min<int64_t>(cdiv(warps_needed, 8), int64_t(d->sm_count) * 8));
+        launch(nvfp4::amax_kernel, dim3(grid), dim3(256), 0, stream, static_cast<const uint16_t *>(X), rows, K, ld,
+               slices, seg, amax_ws, d->status, static_cast<int32_t>(0));
+        g_launches++;
+        return launch_ok();
+    }
+    return NVFP4_OK;
+}
+
+// K1 + K2 for `rows` x K bf16 rows, segment table `seg`.  mode 0: dynamic
+// scale from max|x| (amax words in ws, g written to g_out); mode 1: scale
+// read from g_in.
 int run_quantize(DeviceState *d, const void *X, int64_t rows, int64_t K, int64_t ld, const nvfp4::SegRows &seg,
                  uint8_t *codes, uint8_t *sf, const float *g_in, float *g_out, bool dynamic, uint32_t *amax_ws,
                  cudaStream_t stream, int64_t gate_up_F = 0)
@@ -173,20 +202,8 @@ int run_quantize(DeviceState *d, const void *X, int64_t rows, int64_t K, int64_t
     const int64_t groups = cdiv(K, 64);
     if (rows_pad * groups * 4 >= (int64_t(1) << 31) || K > (int64_t(1) << 30))
         return NVFP4_ERR_UNSUPPORTED_SHAPE;
-    if (dynamic) {
-        if (zero_words(amax_ws, seg.nseg, stream) != NVFP4_OK)
-            return NVFP4_ERR_CUDA;
-        if (rows > 0) {
-            const int64_t slices = amax_slices(rows, K);
-            const int64_t warps_needed = rows * slices;
-            int grid = static_cast<int>(std::min<int64_t>(cdiv(warps_needed, 8), int64_t(d->sm_count) * 8));
-            launch(nvfp4::amax_kernel, dim3(grid), dim3(256), 0, stream, static_cast<const uint16_t *>(X), rows, K, ld,
-                   slices, seg, amax_ws, d->status);
-            g_launches++;
-            if (launch_ok() != NVFP4_OK)
-                return NVFP4_ERR_CUDA;
-        }
-    }
+    if (dynamic && run_amax(d, X, rows, K, ld, seg, amax_ws, stream) != NVFP4_OK)
+        return NVFP4_ERR_CUDA;
     nvfp4::QuantParams p;
     p.X = static_cast<const uint16_t *>(X);
     p.ld = ld;
@@ -1010,20 +1027,11 @@ extern "C" int nvfp4_fp8_kv_calibrate(const void *X, int64_t rows, int64_t cols,
         return NVFP4_ERR_NO_DEVICE;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     uint32_t *amax = static_cast<uint32_t *>(ws);
-    if (zero_words(amax, 1, s) != NVFP4_OK)
+    nvfp4::SegRows seg;
+    nvfp4_segment one = {0, std::max<int64_t>(rows, 1)};
+    check_segments(&one, 1, std::max<int64_t>(rows, 1), &seg);
+    if (run_amax(d, X, cols > 0 ? rows : 0, cols, ldx, seg, amax, s) != NVFP4_OK)
         return NVFP4_ERR_CUDA;
-    if (rows > 0 && cols > 0) {
-        nvfp4::SegRows seg;
-        nvfp4_segment one = {0, rows};
-        check_segments(&one, 1, rows, &seg);
-        const int64_t slices = amax_slices(rows, cols);
-        const int grid = static_cast<int>(std::min<int64_t>(cdiv(rows * slices, 8), int64_t(d->sm_count) * 8));
-        launch(nvfp4::amax_kernel, dim3(grid), dim3(256), 0, s, static_cast<const uint16_t *>(X), rows, cols, ldx, slices,
-               seg, amax, d->status);
-        g_launches++;
-        if (launch_ok() != NVFP4_OK)
-            return NVFP4_ERR_CUDA;
-    }
     launch(nvfp4::kv::kv_scale_kernel, dim3(1), dim3(32), 0, s, amax, scale);
     g_launches++;
     return launch_ok();

@@ -84,14 +84,16 @@ __global__ void zero_words_kernel(uint32_t *__restrict__ words, int32_t n)
 }
 
 // amax_bits[seg] = max over the segment's rows of the bf16 magnitude bits
-// (the float max|x| is amax_bits << 16).  amax_bits must be zero on entry.
+// (the float max|x| is amax_bits << 16).  amax_bits must be zero on entry,
+// except with `direct` (a launch of one CTA), where the CTA stores its maxima.
 // Each row is cut into `slices` contiguous ranges of 16-byte chunks, one warp
 // per (row, range): one range per row when there are rows enough to fill the
 // GPU, several when there are few (decode-sized inputs), so that a short
 // input is read by many warps at once instead of a few long loops.
-__global__ void __launch_bounds__(256) amax_kernel(const uint16_t *__restrict__ X, int64_t rows, int64_t K,
-                                                   int64_t ld, int64_t slices, SegRows seg,
-                                                   uint32_t *__restrict__ amax_bits, uint32_t *__restrict__ status)
+__global__ void __launch_bounds__(1024) amax_kernel(const uint16_t *__restrict__ X, int64_t rows, int64_t K,
+                                                    int64_t ld, int64_t slices, SegRows seg,
+                                                    uint32_t *__restrict__ amax_bits, uint32_t *__restrict__ status,
+                                                    int32_t direct)
 {
     grid_dep_wait();
     grid_dep_launch_dependents();
@@ -134,7 +136,9 @@ __global__ void __launch_bounds__(256) amax_kernel(const uint16_t *__restrict__ 
     __syncthreads();
     if (threadIdx.x < seg.nseg) {
         const uint32_t v = s_max[threadIdx.x];
-        if (v != 0)
+        if (direct)
+            amax_bits[threadIdx.x] = v;
+        else if (v != 0)
             atomicMax(&amax_bits[threadIdx.x], v);
         if (v >= 0x7F80u)  // Inf or NaN magnitude
             atomicOr(status, kStatusNonFinite);

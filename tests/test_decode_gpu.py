@@ -76,22 +76,26 @@ def test_decode_linear_matches_oracle(M, N, K, widths):
 
 def test_split_sum_is_its_own_launch():
     """K = 5120 at N = 5120 splits K (one more launch adds the partials);
-    K = 256 has one stage and cannot split."""
+    K = 256 has one stage and cannot split.  Counted as the linear's launches
+    minus those of quantizing the same input."""
     W, _ = _weight(5120, 5120, None, 1)
     qw = ops.quantize_weights(W.to(DEV))
     qs = ops.quantize_weights(W[:, :256].contiguous().to(DEV))
 
-    def launches(M, K, q):
+    def gemm_launches(M, K, q):
         X = wl.activation_normal(M, K, 1).to(DEV)
         ops.linear(X, q)
+        ops.quantize_act(X)
         torch.cuda.synchronize()
         n0 = ops.launch_count()
         ops.linear(X, q)
-        return ops.launch_count() - n0
+        n1 = ops.launch_count()
+        ops.quantize_act(X)
+        return (n1 - n0) - (ops.launch_count() - n1)
 
-    unsplit = launches(16, 256, qs)
-    assert launches(1, 5120, qw) == unsplit + 1
-    assert launches(16, 5120, qw) == unsplit + 1
+    assert gemm_launches(16, 256, qs) == 1
+    assert gemm_launches(1, 5120, qw) == 2
+    assert gemm_launches(16, 5120, qw) == 2
     assert ops.get_status() == 0
 
 
