@@ -76,6 +76,11 @@ struct Params {
     int32_t M, N, K;
     int32_t num_m, num_n, num_tiles;
     int32_t pair_m, pair_n, pair_tiles;  // 256 x 256 tiles of the CTA-pair kernel
+    // Bytes of the activation box the single-CTA kernel loads per stage: all
+    // 128 rows, or only round_up(M, 8) of them when M < 128 (decode).  The
+    // stage's other rows keep stale codes; they meet only the zero or stale
+    // scales of rows >= M and feed accumulator rows that are never stored.
+    uint32_t a_box_bytes;
     // Split-K (single-CTA kernel, small M): work item t covers tile
     // t % num_tiles over the K steps of split t / num_tiles; with splits > 1
     // the epilogue writes alpha * acc as fp32 to partial[split][M][N] and a
@@ -381,7 +386,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     const uint32_t bar = smem_u32(&sm->full[stage]);
                     const int32_t sf_x = kt * KB_PER_STAGE * (SF_TILE / 8);
                     if (!w_side) {
-                        mbar_arrive_expect_tx(bar, A_BYTES + p.sf_box_bytes);
+                        mbar_arrive_expect_tx(bar, p.a_box_bytes + p.sf_box_bytes);
                         tma_load_2d(a_smem(stage), &tmA, kt * BK_BYTES, m0, bar);
                         tma_load_2d(sfa_smem(stage), &tmSFA, sf_x, m_blk, bar);
                     } else {

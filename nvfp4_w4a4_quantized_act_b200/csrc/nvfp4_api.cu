@@ -362,7 +362,9 @@ int run_gemm(DeviceState *d, const uint8_t *a_codes, const uint8_t *a_sf, const 
     uint32_t sf_box = 0, sf_box_b = 0;
     // CTA pairs (256-row tiles) once A has more than one 128-row block
     const bool use_pair = (M > BM) && !(flags & NVFP4_SINGLE_CTA);
-    if (make_codes_map(&tmA, a_codes, M, K, BM) != NVFP4_OK ||
+    // the single-CTA kernel loads only the rows a small M has (multiple of 8: one swizzle atom)
+    const uint32_t a_rows = (!use_pair && M < BM) ? static_cast<uint32_t>(round_up(M, 8)) : static_cast<uint32_t>(BM);
+    if (make_codes_map(&tmA, a_codes, M, K, a_rows) != NVFP4_OK ||
         make_codes_map(&tmB, w_codes, N, K, use_pair ? 128u : static_cast<uint32_t>(BN)) != NVFP4_OK ||
         make_sf_map(&tmSFA, a_sf, cdiv(M, 128), K / 64, 1, &sf_box) != NVFP4_OK ||
         make_sf_map(&tmSFB, w_sf, n_row_tiles, K / 64, sfb_rows, &sf_box_b) != NVFP4_OK)
@@ -375,6 +377,7 @@ int run_gemm(DeviceState *d, const uint8_t *a_codes, const uint8_t *a_sf, const 
     p.num_m = static_cast<int32_t>(cdiv(M, BM));
     p.num_n = static_cast<int32_t>(cdiv(N, BN));
     p.num_tiles = p.num_m * p.num_n;
+    p.a_box_bytes = a_rows * BK_BYTES;
     p.pair_m = static_cast<int32_t>(cdiv(M, pair::PAIR_M));
     p.pair_n = static_cast<int32_t>(cdiv(N, pair::PAIR_N));
     p.pair_tiles = p.pair_m * p.pair_n;
