@@ -194,9 +194,11 @@ int run_amax(DeviceState *d, const void *X, int64_t rows, int64_t K, int64_t ld,
 // K1 + K2 for `rows` x K bf16 rows, segment table `seg`.  mode 0: dynamic
 // scale from max|x| (amax words in ws, g written to g_out); mode 1: scale
 // read from g_in.
+// zero_word, if given, is cleared by the quantize kernel (for the kernel that
+// follows on the stream).
 int run_quantize(DeviceState *d, const void *X, int64_t rows, int64_t K, int64_t ld, const nvfp4::SegRows &seg,
                  uint8_t *codes, uint8_t *sf, const float *g_in, float *g_out, bool dynamic, uint32_t *amax_ws,
-                 cudaStream_t stream, int64_t gate_up_F = 0)
+                 cudaStream_t stream, int64_t gate_up_F = 0, uint32_t *zero_word = nullptr)
 {
     const int64_t rows_pad = round_up(rows, 128);
     const int64_t groups = cdiv(K, 64);
@@ -219,6 +221,7 @@ int run_quantize(DeviceState *d, const void *X, int64_t rows, int64_t K, int64_t
     p.codes = codes;
     p.sf = sf;
     p.gate_up_F = static_cast<int32_t>(gate_up_F);
+    p.zero = zero_word;
     const int64_t threads = rows_pad * groups * 4;
     int grid = static_cast<int>(std::min<int64_t>(std::max<int64_t>(cdiv(threads, 256), 1), int64_t(d->sm_count) * 16));
     launch(nvfp4::quantize_kernel, dim3(grid), dim3(256), 0, stream, p);
@@ -976,16 +979,17 @@ extern "C" int nvfp4_linear_swiglu(const void *X, int64_t M, int64_t K, const ui
     nvfp4::SegRows one_seg;
     nvfp4_segment one = {0, M};
     check_segments(&one, 1, M, &one_seg);
-    // X -> NVFP4 (dynamic scale unless a calibrated one is supplied)
-    rc = run_quantize(d, X, M, K, K, one_seg, a_codes, a_sf, g_a, g_a, (flags & NVFP4_STATIC_SCALE) == 0, amax, s);
+    // X -> NVFP4 (dynamic scale unless a calibrated one is supplied); the
+    // quantize kernel also clears max|h| for the GEMM's epilogue
+    rc = run_quantize(d, X, M, K, K, one_seg, a_codes, a_sf, g_a, g_a, (flags & NVFP4_STATIC_SCALE) == 0, amax, s, 0,
+                      h_amax);
     if (rc != NVFP4_OK)
         return rc;
     // gate/up GEMM with the SwiGLU epilogue -> h (bf16) and max|h|
-    if (zero_words(h_amax, 1, s) != NVFP4_OK)
-        return NVFP4_ERR_CUDA;
     nvfp4::SegRows gu;
     const nvfp4_segment two[2] = {{0, F}, {F, 2 * F}};
     check_segments(two, 2, 2 * F, &gu);
+    // the GEMM follows this call's own quantize kernel, which does not write W
     rc = run_gemm(d, a_codes, a_sf, g_a, M, K, w_codes, w_sf, 2 * F, gu, g_w, h, flags & NVFP4_SINGLE_CTA, s, h_amax,
                   nullptr, true);
     if (rc != NVFP4_OK)

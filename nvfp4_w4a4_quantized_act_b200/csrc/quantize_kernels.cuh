@@ -162,6 +162,7 @@ struct QuantParams {
     uint8_t *codes;          // [rows, K/2]
     uint8_t *sf;             // swizzled scale tiles
     int32_t gate_up_F;       // > 0: rows are [gate F | up F]; stored interleaved in 128-row blocks
+    uint32_t *zero = nullptr;  // one word block 0 clears (the next GEMM's max|h|), or null
 };
 
 // Stored row of input row r.  With a gate/up pair of F rows each, block b of
@@ -239,6 +240,8 @@ __global__ void __launch_bounds__(256) quantize_kernel(const QuantParams p)
 {
     grid_dep_wait();
     grid_dep_launch_dependents();
+    if (p.zero != nullptr && blockIdx.x == 0 && threadIdx.x == 0)
+        *p.zero = 0;
     __shared__ float s_g[kMaxSeg], s_rg[kMaxSeg];
     __shared__ int s_gok[kMaxSeg];
     if (threadIdx.x < p.seg.nseg) {
