@@ -509,20 +509,22 @@ def fp8_kv_roofline(pk, pk_kind):
 def decode_roofline(stack, pk, pk_kind, token_counts=(1, 16, 64, 128)):
     """Decode steps through the same 64-layer stack: M new tokens per step
     (M <= 128 runs the split-K GEMM), every linear through the public calls
-    (nvfp4_linear_fused; nvfp4_linear_swiglu for gate/up; the down projection
-    re-quantizes h through nvfp4_linear_fused).  A step streams every NVFP4
+    (nvfp4_linear_fused; nvfp4_linear_swiglu for gate/up, whose quantized h
+    feeds the down projection through nvfp4_gemm_prequant_ws).  A step streams every NVFP4
     weight once (13.4 GB, far above L2), so it is bound by HBM: the figure is
     weight bytes per step / step time.  Each step is one CUDA graph of 256
     linears (captured once per M, replayed)."""
     from nvfp4_w4a4_quantized_act_b200 import ops
     dev = stack.X.device
     wbytes = sum(qw.codes.numel() + qw.sf.numel() for qs in stack.weights for qw in qs)
-    res = {"kernel": "split-K linear chain (amax + quantize + gemm_nvf4_kernel split-K + split sum) per linear",
+    res = {"kernel": "split-K linear chain (amax + quantize + gemm_nvf4_kernel split-K + split sum) per linear; "
+                     "gate/up with SwiGLU, down on its quantized h",
            "bound": "hbm", "unit": "GB/s", "peak": pk["hbm_gbs"], "peak_basis": pk_kind,
            "weight_bytes_per_step": int(wbytes), "linears_per_step": 256, "steps": {}}
     for M in token_counts:
         X, X2, Y = stack.X[:M], stack.X2[:M], stack.Y[:M]
-        ws_bytes = max(ops.workspace_bytes(M, lin.N, lin.K, len(lin.segments))
+        ws_bytes = max(max(ops.workspace_bytes(M, lin.N, lin.K, len(lin.segments)),
+                           ops.gemm_workspace_bytes(M, lin.N, lin.K))
                        for _, lins in stack.layers for lin in lins)
         ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
         h = torch.empty((M, 17408), dtype=torch.bfloat16, device=dev)
@@ -537,7 +539,7 @@ def decode_roofline(stack, pk, pk_kind, token_counts=(1, 16, 64, 128)):
                     if lin.name == "gate_up":
                         ops.linear_swiglu(X2, qw, h=h, h_codes=hc, h_sf=hsf, g_h=gh, ws=ws)
                     elif lin.name == "down":
-                        ops.linear_fused(h, qw, out=outs[5120], ws=ws)
+                        ops.gemm_prequant(hc, hsf, gh, M, lin.K, qw, out=outs[5120], ws=ws)
                     else:
                         src = Y if lin.name in ("gdn_out", "attn_o") else X
                         if lin.N not in outs:

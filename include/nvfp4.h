@@ -157,6 +157,20 @@ int nvfp4_gemm_prequant(const uint8_t *a_codes, const uint8_t *a_sf, const float
                         const nvfp4_segment *segs, const float *g_w, int nseg,
                         void *out, unsigned flags, void *stream);
 
+/* nvfp4_gemm_prequant with a workspace: for M <= 128 the GEMM may divide K
+ * among several CTAs (split-K, as nvfp4_linear_fused does; the fp32 partials
+ * live in ws and are added in a fixed order).  ws: at least
+ * nvfp4_gemm_workspace_bytes(M, N, K) bytes, 16-byte aligned (the size is 0
+ * where no split is used; ws may then be NULL).  Use it where the activation
+ * is already quantized at decode sizes, e.g. the down projection after
+ * nvfp4_linear_swiglu. */
+size_t nvfp4_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
+int nvfp4_gemm_prequant_ws(const uint8_t *a_codes, const uint8_t *a_sf, const float *g_a,
+                           int64_t M, int64_t K,
+                           const uint8_t *w_codes, const uint8_t *w_sf, int64_t N,
+                           const nvfp4_segment *segs, const float *g_w, int nseg,
+                           void *out, unsigned flags, void *ws, size_t ws_bytes, void *stream);
+
 /* Fused-module linear: quantize X (as nvfp4_quantize_act, into the
  * workspace) then nvfp4_gemm_prequant against a fused weight whose rows are
  * split into nseg modules, each with its own global scale g_w[m].

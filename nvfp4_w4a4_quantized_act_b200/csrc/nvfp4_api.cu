@@ -495,6 +495,56 @@ size_t linear_partial_bytes(int64_t M, int64_t N, int64_t K)
     return S > 1 ? static_cast<size_t>(S) * static_cast<size_t>(M) * static_cast<size_t>(N) * 4 : 0;
 }
 
+// nvfp4_gemm_prequant with an optional workspace for split-K partial sums
+// (ws == nullptr: never split).
+int gemm_prequant_impl(const uint8_t *a_codes, const uint8_t *a_sf, const float *g_a, int64_t M, int64_t K,
+                       const uint8_t *w_codes, const uint8_t *w_sf, int64_t N, const nvfp4_segment *segs,
+                       const float *g_w, int nseg, void *out, unsigned flags, void *ws, size_t ws_bytes,
+                       void *stream)
+{
+    if ((flags & ~(NVFP4_STATIC_SCALE | NVFP4_OUT_FP32 | NVFP4_DEBUG_INJECT_STALL | NVFP4_SINGLE_CTA)) != 0)
+        return NVFP4_ERR_INVALID_ARG;
+    int rc = check_gemm_shape(M, N, K);
+    if (rc != NVFP4_OK)
+        return rc;
+    {
+        nvfp4::SegRows seg0;
+        rc = check_segments(segs, nseg, N, &seg0);
+        if (rc != NVFP4_OK)
+            return rc;
+    }
+    if (M == 0 || N == 0)
+        return NVFP4_OK;
+    if (a_codes == nullptr || a_sf == nullptr || g_a == nullptr || w_codes == nullptr || w_sf == nullptr ||
+        g_w == nullptr || out == nullptr)
+        return NVFP4_ERR_INVALID_ARG;
+    if (!aligned16(a_codes) || !aligned16(a_sf) || !aligned16(w_codes) || !aligned16(w_sf) ||
+        (reinterpret_cast<uintptr_t>(g_a) & 3u) || (reinterpret_cast<uintptr_t>(g_w) & 3u) ||
+        (reinterpret_cast<uintptr_t>(out) & ((flags & NVFP4_OUT_FP32) ? 3u : 1u)))
+        return NVFP4_ERR_MISALIGNED;
+    nvfp4::SegRows seg;
+    rc = check_segments(segs, nseg, N, &seg);
+    if (rc != NVFP4_OK)
+        return rc;
+    float *partial = nullptr;
+    if (ws != nullptr) {
+        const size_t need = linear_partial_bytes(M, N, K);
+        if (ws_bytes < need)
+            return NVFP4_ERR_WORKSPACE;
+        if (!aligned16(ws))
+            return NVFP4_ERR_MISALIGNED;
+        if (need > 0)
+            partial = static_cast<float *>(ws);
+    }
+    DeviceState *d = device_state();
+    if (d == nullptr)
+        return NVFP4_ERR_CUDA;
+    if (!d->supported)
+        return NVFP4_ERR_NO_DEVICE;
+    return run_gemm(d, a_codes, a_sf, g_a, M, K, w_codes, w_sf, N, seg, g_w, out, flags,
+                    static_cast<cudaStream_t>(stream), nullptr, partial);
+}
+
 }  // namespace
 
 // ======================================================================== C ABI
@@ -591,37 +641,24 @@ int nvfp4_gemm_prequant(const uint8_t *a_codes, const uint8_t *a_sf, const float
                         const uint8_t *w_codes, const uint8_t *w_sf, int64_t N, const nvfp4_segment *segs,
                         const float *g_w, int nseg, void *out, unsigned flags, void *stream)
 {
-    if ((flags & ~(NVFP4_STATIC_SCALE | NVFP4_OUT_FP32 | NVFP4_DEBUG_INJECT_STALL | NVFP4_SINGLE_CTA)) != 0)
-        return NVFP4_ERR_INVALID_ARG;
-    int rc = check_gemm_shape(M, N, K);
-    if (rc != NVFP4_OK)
-        return rc;
-    {
-        nvfp4::SegRows seg0;
-        rc = check_segments(segs, nseg, N, &seg0);
-        if (rc != NVFP4_OK)
-            return rc;
-    }
-    if (M == 0 || N == 0)
-        return NVFP4_OK;
-    if (a_codes == nullptr || a_sf == nullptr || g_a == nullptr || w_codes == nullptr || w_sf == nullptr ||
-        g_w == nullptr || out == nullptr)
-        return NVFP4_ERR_INVALID_ARG;
-    if (!aligned16(a_codes) || !aligned16(a_sf) || !aligned16(w_codes) || !aligned16(w_sf) ||
-        (reinterpret_cast<uintptr_t>(g_a) & 3u) || (reinterpret_cast<uintptr_t>(g_w) & 3u) ||
-        (reinterpret_cast<uintptr_t>(out) & ((flags & NVFP4_OUT_FP32) ? 3u : 1u)))
-        return NVFP4_ERR_MISALIGNED;
-    nvfp4::SegRows seg;
-    rc = check_segments(segs, nseg, N, &seg);
-    if (rc != NVFP4_OK)
-        return rc;
-    DeviceState *d = device_state();
-    if (d == nullptr)
-        return NVFP4_ERR_CUDA;
-    if (!d->supported)
-        return NVFP4_ERR_NO_DEVICE;
-    return run_gemm(d, a_codes, a_sf, g_a, M, K, w_codes, w_sf, N, seg, g_w, out, flags,
-                    static_cast<cudaStream_t>(stream));
+    return gemm_prequant_impl(a_codes, a_sf, g_a, M, K, w_codes, w_sf, N, segs, g_w, nseg, out, flags, nullptr, 0,
+                              stream);
+}
+
+size_t nvfp4_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K)
+{
+    if (M < 0 || N < 0 || K <= 0 || K % 64 != 0)
+        return 0;
+    return linear_partial_bytes(M, N, K);
+}
+
+int nvfp4_gemm_prequant_ws(const uint8_t *a_codes, const uint8_t *a_sf, const float *g_a, int64_t M, int64_t K,
+                           const uint8_t *w_codes, const uint8_t *w_sf, int64_t N, const nvfp4_segment *segs,
+                           const float *g_w, int nseg, void *out, unsigned flags, void *ws, size_t ws_bytes,
+                           void *stream)
+{
+    return gemm_prequant_impl(a_codes, a_sf, g_a, M, K, w_codes, w_sf, N, segs, g_w, nseg, out, flags, ws, ws_bytes,
+                              stream);
 }
 
 int nvfp4_linear_fused(const void *X, int64_t M, int64_t K, const uint8_t *w_codes, const uint8_t *w_sf, int64_t N,

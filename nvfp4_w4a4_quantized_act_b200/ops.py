@@ -32,6 +32,7 @@ STATUS_NAMES = {
 EXPORTED = [
     "nvfp4_sf_bytes", "nvfp4_quant_workspace_bytes", "nvfp4_workspace_bytes", "nvfp4_linear_act_scale_offset",
     "nvfp4_quantize_weights", "nvfp4_quantize_act", "nvfp4_gemm_prequant", "nvfp4_linear_fused",
+    "nvfp4_gemm_workspace_bytes", "nvfp4_gemm_prequant_ws",
     "nvfp4_linear", "nvfp4_swiglu_quantize", "nvfp4_get_status", "nvfp4_status_string",
     "nvfp4_device_supported", "nvfp4_launch_count", "nvfp4_linear_fused_noalloc",
     "nvfp4_quantize_weights_gated", "nvfp4_linear_swiglu", "nvfp4_gemm_prequant_swiglu",
@@ -69,6 +70,9 @@ def lib() -> ctypes.CDLL:
         "nvfp4_linear_act_scale_offset": (sz, []),
         "nvfp4_quantize_weights": (ctypes.c_int, [vp, i64, i64, i64, segp, ctypes.c_int, u8p, u8p, fp, vp, sz, vp]),
         "nvfp4_quantize_act": (ctypes.c_int, [vp, i64, i64, i64, u8p, u8p, fp, ctypes.c_uint, vp, sz, vp]),
+        "nvfp4_gemm_workspace_bytes": (sz, [i64, i64, i64]),
+        "nvfp4_gemm_prequant_ws": (ctypes.c_int, [u8p, u8p, fp, i64, i64, u8p, u8p, i64, segp, fp, ctypes.c_int,
+                                                  vp, ctypes.c_uint, vp, sz, vp]),
         "nvfp4_gemm_prequant": (ctypes.c_int, [u8p, u8p, fp, i64, i64, u8p, u8p, i64, segp, fp, ctypes.c_int, vp,
                                                ctypes.c_uint, vp]),
         "nvfp4_linear_fused": (ctypes.c_int, [vp, i64, i64, u8p, u8p, i64, segp, fp, ctypes.c_int, vp,
@@ -210,15 +214,26 @@ def quantize_act(X: torch.Tensor, g_a: torch.Tensor | None = None, static_scale:
     return codes[: M * K // 2].view(M, K // 2), sf, g_a
 
 
+def gemm_workspace_bytes(M: int, N: int, K: int) -> int:
+    return int(lib().nvfp4_gemm_workspace_bytes(M, N, K))
+
+
 def gemm_prequant(a_codes, a_sf, g_a, M: int, K: int, w: QuantizedWeight, out=None, out_fp32=False, stream=None,
-                  debug_flags: int = 0):
-    """nvfp4_gemm_prequant on already-quantized activations."""
+                  debug_flags: int = 0, ws=None):
+    """nvfp4_gemm_prequant on already-quantized activations; with a workspace
+    (ws, gemm_workspace_bytes(M, N, K) bytes) nvfp4_gemm_prequant_ws, which may
+    split K at decode sizes."""
     _require_cuda(a_codes, a_sf, g_a)
     dt = torch.float32 if out_fp32 else torch.bfloat16
     if out is None:
         out = torch.empty((M, w.N), dtype=dt, device=a_codes.device)
     arr, n = _segs(w.segments)
     flags = (NVFP4_OUT_FP32 if out_fp32 else 0) | debug_flags
+    if ws is not None:
+        _check(lib().nvfp4_gemm_prequant_ws(_p(a_codes), _p(a_sf), _p(g_a), M, K, _p(w.codes), _p(w.sf), w.N, arr,
+                                            _p(w.g_w), n, _p(out), flags, _p(ws), ws.numel(), _stream(stream)),
+               "nvfp4_gemm_prequant_ws")
+        return out
     _check(lib().nvfp4_gemm_prequant(_p(a_codes), _p(a_sf), _p(g_a), M, K, _p(w.codes), _p(w.sf), w.N, arr,
                                      _p(w.g_w), n, _p(out), flags, _stream(stream)), "nvfp4_gemm_prequant")
     return out

@@ -75,6 +75,20 @@ def test_decode_workspace_holds_split_partials(L, M, N, K, splits):
         assert ops.workspace_bytes(M, N, K) == act
     else:
         assert ops.workspace_bytes(M, N, K) == -(-act // 256) * 256 + splits * M * N * 4
+    # the pre-quantized GEMM's workspace is the partials alone
+    assert ops.gemm_workspace_bytes(M, N, K) == (splits * M * N * 4 if splits > 1 else 0)
+
+
+def test_gemm_workspace_argument_errors(L):
+    fake = ctypes.c_void_p(1 << 20)
+    one = _segarr([(0, 5120)])
+    need = ops.gemm_workspace_bytes(16, 5120, 5120)
+    assert need > 0 and ops.gemm_workspace_bytes(16, 5120, 96) == 0
+    assert L.nvfp4_gemm_prequant_ws(fake, fake, fake, 16, 5120, fake, fake, 5120, one, fake, 1, fake, 0, fake,
+                                    need - 4, None) == 7
+    mis = ctypes.c_void_p((1 << 20) + 8)
+    assert L.nvfp4_gemm_prequant_ws(fake, fake, fake, 16, 5120, fake, fake, 5120, one, fake, 1, fake, 0, mis,
+                                    need, None) == 3
 
 
 def _segarr(pairs):

@@ -72,6 +72,11 @@ def test_decode_linear_matches_oracle(M, N, K, widths):
     plain = host(ops.gemm_prequant(c_ws, sf_ws, g_ws, M, K, qw, out_fp32=True))
     assert ops.get_status() == 0
     check_gemm(plain[:, cols], C, B, "unsplit")
+    # the workspace form splits like the linear: the same bits on the same operands
+    gws = torch.empty(max(ops.gemm_workspace_bytes(M, N, K), 16), dtype=torch.uint8, device=DEV)
+    pre = host(ops.gemm_prequant(c_ws, sf_ws, g_ws, M, K, qw, out_fp32=True, ws=gws))
+    assert ops.get_status() == 0
+    assert np.array_equal(pre, out32)
 
 
 def test_split_sum_is_its_own_launch():
