@@ -3,8 +3,8 @@
  * (libnvfp4.so).
  *
  * The method: every linear layer of a hybrid LLM runs with 4-bit weights and
- * 4-bit activations in NVFP4, i.e. E2M1 values with one E4M3 scale per
- * 16-element block ("NVFP4 W4A4 quantization compresses 27B hybrid models",
+ * 4-bit activations in NVFP4, i.e. E2M1 codes where each group of 16
+ * consecutive codes shares one E4M3 scale ("NVFP4 W4A4 quantization compresses 27B hybrid models",
  * thevalue.engineering, section "Challenging the Recurrence Fragility
  * Assumption"; "Why Gated DeltaNet Survives 4-Bit Quantization", kipquest.com,
  * "The abstract" and "The deep dive").  Checkpoints are calibrated per module,
@@ -124,8 +124,8 @@ size_t nvfp4_workspace_bytes(int64_t M, int64_t N, int64_t K, int nseg);
  * rows into modules; each module m gets its own dynamic global scale
  * g_w[m] = amax_m/2688 (written to the device array g_w[nseg]).
  * Outputs: codes [N, K/2], sf (nvfp4_sf_bytes(N, K) bytes).  K % 16 == 0.
- * Passages: per-module-calibrated NVFP4 checkpoints (kipquest.com, "The
- * abstract"); weights rounded after training rather than trained under
+ * Passages: checkpoints whose modules were each calibrated with their own
+ * scale (kipquest.com, "The abstract"); weights rounded after training rather than trained under
  * quantization (same page, "The deep dive"). */
 int nvfp4_quantize_weights(const void *W, int64_t N, int64_t K, int64_t ldw,
                            const nvfp4_segment *segs, int nseg,
@@ -149,8 +149,8 @@ int nvfp4_quantize_act(const void *X, int64_t M, int64_t K, int64_t ldx,
  * accumulated in fp32 on the tensor cores.  out is [M, N] row-major, bf16
  * (round to nearest even) or fp32 with NVFP4_OUT_FP32.  K % 64 == 0.
  * g_a: device, 1 float; g_w: device, nseg floats; segs: host.
- * Passage: kernels that fuse per-module-calibrated modules into one GEMM and
- * the global-scale repair (kipquest.com, "The abstract", "The deep dive"). */
+ * Passage: serving separately calibrated modules through one fused GEMM,
+ * and the global-scale repair (kipquest.com, "The abstract", "The deep dive"). */
 int nvfp4_gemm_prequant(const uint8_t *a_codes, const uint8_t *a_sf, const float *g_a,
                         int64_t M, int64_t K,
                         const uint8_t *w_codes, const uint8_t *w_sf, int64_t N,

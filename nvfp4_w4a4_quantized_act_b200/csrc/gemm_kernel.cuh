@@ -8,8 +8,8 @@
 // The block-scaled product runs on the tensor cores without emulation ("Why
 // Gated DeltaNet Survives 4-Bit Quantization", kipquest.com, "The deep
 // dive"); applying each module's own FP32 global scale to its columns is the
-// repair of the global-scale mismatch that appears when per-module-calibrated
-// checkpoints are served by a kernel that fuses those modules into one GEMM
+// repair of the global-scale mismatch: modules calibrated one by one, then
+// run as a single fused GEMM under one scale, give wrong outputs
 // (same page, "The abstract" and "The deep dive").
 //
 // Tile 128 x 256 (x 256 of K per pipeline stage), one CTA per SM, 12 warps:

@@ -13,8 +13,8 @@
 //  swiglu_kernel    h = bf16(silu(gate) * up) for a fused gate/up output, plus
 //                   max|h| for its dynamic global scale.
 //
-// Format and scale conventions: NVFP4 = E2M1 values with an E4M3 scale per
-// 16-element block ("NVFP4 W4A4 quantization compresses 27B hybrid models",
+// Format and scale conventions: NVFP4 = E2M1 codes, each group of 16
+// consecutive codes sharing one E4M3 scale ("NVFP4 W4A4 quantization compresses 27B hybrid models",
 // thevalue.engineering, "Challenging the Recurrence Fragility Assumption"),
 // one FP32 global scale per calibrated module ("Why Gated DeltaNet Survives
 // 4-Bit Quantization", kipquest.com, "The abstract").

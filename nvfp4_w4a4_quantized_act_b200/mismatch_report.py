@@ -2,9 +2,10 @@
 weights through one fused GEMM with a single global scale does to each
 module's outputs, and what each repair leaves.
 
-The pages describe the fault: checkpoints calibrated per module, served by
-kernels that fuse those modules into one matrix multiply, come out wrong (the
-gates are corrupted with no error raised) -- kipquest.com, "Why Gated DeltaNet Survives
+The pages describe the fault: when each module carries its own calibrated
+global scale and a serving kernel runs the modules as one GEMM under a single
+scale, the outputs go wrong without any error showing, and the gates are the
+modules they name as damaged -- kipquest.com, "Why Gated DeltaNet Survives
 4-Bit Quantization", sections "The abstract" and "The deep dive".  They give
 no error figures; this measures them on synthetic tensors shaped like the GDN
 input projection (q, k, v, z, b, a: N = 16480 in six modules whose weight

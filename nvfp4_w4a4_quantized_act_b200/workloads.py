@@ -7,7 +7,7 @@ Shapes follow the model the paper quantizes: a 48 Gated-DeltaNet / 16
 attention hybrid with hidden size 5120 and MLP width 17408 ("Why Gated
 DeltaNet Survives 4-Bit Quantization", kipquest.com, "The abstract" and "The
 deep dive").  Outliers follow the deep dive's remark that the residual stream
-has hot channels about a hundred times the median.
+has a few channels whose magnitude is about 100x the median.
 
 Every generator is seeded; values are drawn in fp32/fp64 with numpy's PCG64
 (or torch's CUDA generator for the large stack weights) and rounded to bf16

@@ -8,7 +8,8 @@ The arithmetic lives in ``nvfp4_oracle.c`` (plain C, fp32 steps written out
 one operation at a time, fp64 GEMM); this module only marshals numpy arrays.
 It follows the pages on the method:
 
-* NVFP4 = E2M1 4-bit values with an E4M3 scale per 16-element block
+* NVFP4 = 4-bit E2M1 codes, each group of 16 consecutive codes sharing one
+  E4M3 scale
   ("NVFP4 W4A4 quantization compresses 27B hybrid models", thevalue.engineering,
   section "Challenging the Recurrence Fragility Assumption"; "Quantizing All
   Layers Reveals Recurrent Memory Is Robust", freegardner.com, section "Block

@@ -5,18 +5,18 @@
  * the product path.  It shares no source with the CUDA library.
  *
  * What it follows:
- *  - "NVFP4 pairs E2M1 4-bit values with an E4M3 scale per 16-element block"
- *    (thevalue.engineering, "NVFP4 W4A4 quantization compresses 27B hybrid
- *    models", section "Challenging the Recurrence Fragility Assumption"); the
- *    same 16-element grouping is described on freegardner.com, "Quantizing
- *    All Layers Reveals Recurrent Memory Is Robust", section "Block Scaling
- *    and the Geography of Outliers", and in the kipquest.com paper page
- *    "Why Gated DeltaNet Survives 4-Bit Quantization", section "The deep
- *    dive" (one shared scale per sixteen-element block).
+ *  - NVFP4 elements are 4-bit E2M1 codes; every 16 consecutive codes share
+ *    one E4M3 scale (thevalue.engineering, "NVFP4 W4A4 quantization
+ *    compresses 27B hybrid models", section "Challenging the Recurrence
+ *    Fragility Assumption").  The 16-element grouping is also on
+ *    freegardner.com, "Quantizing All Layers Reveals Recurrent Memory Is
+ *    Robust", section "Block Scaling and the Geography of Outliers", and on
+ *    the kipquest.com paper page "Why Gated DeltaNet Survives 4-Bit
+ *    Quantization", section "The deep dive".
  *  - W4A4: weights and activations both in NVFP4 (kipquest.com, "The
  *    abstract").
- *  - One FP32 global scale per module ("per-module-calibrated NVFP4
- *    checkpoints", kipquest.com, "The abstract" and "The deep dive").
+ *  - Each calibrated module carries its own FP32 global scale (kipquest.com,
+ *    "The abstract" and "The deep dive").
  *
  * Readings where the pages are silent (each is listed in the design notes):
  *  - global scale g = fl32(amax / 2688), 2688 = 6 * 448; g = 1 if amax == 0.
@@ -335,9 +335,9 @@ void oracle_swiglu(const uint16_t *gate_up, int64_t rows, int64_t F, int64_t ld,
 
 /* --------------------------------------------- FP8 KV-cache quantization */
 /*
- * The attention KV cache in FP8 with a calibrated per-tensor scale: "ship the
- * calibrated KV-cache scales", which are "performance-free" when calibrated
- * (freegardner.com, "Quantizing All Layers Reveals Recurrent Memory Is
+ * The attention KV cache in FP8 with a calibrated per-tensor scale.  The pages
+ * recommend shipping calibrated cache scales and report that, calibrated,
+ * they cost no accuracy (freegardner.com, "Quantizing All Layers Reveals Recurrent Memory Is
  * Robust", section "The Calibrated Cache That Ships for Free";
  * thevalue.engineering, "NVFP4 W4A4 quantization compresses 27B hybrid
  * models", section "Efficiency Gains and Serving Optimization"; the
