@@ -275,6 +275,36 @@ def test_sf_layout_is_bijection_of_512_byte_tiles():
             assert [oracle.sf_offset(r, c, K) for c in range(4)] == [base + i for i in range(4)]
 
 
+def _documented_sf_positions(rows, K):
+    """Byte position of every logical scale (r, c) in the block-scaled MMA's
+    scale layout, built the way NVIDIA's cuBLAS documentation describes it
+    (section "1D Block Scaling Factors Layout"): pad the [rows, K/16] scale
+    matrix to whole 128 x 4 tiles; store the tiles one after another, K-tiles
+    fastest, 512 bytes each; inside a tile, split the 128 rows into four
+    groups of 32 and interleave them, so that 16 consecutive bytes hold the
+    4 scales of rows j, j+32, j+64 and j+96.  Expressed here with array
+    reshapes, not with the oracle's modular arithmetic."""
+    rpad = (rows + 127) // 128 * 128
+    cpad = (K // 16 + 3) // 4 * 4
+    idx = np.arange(rpad * cpad).reshape(rpad, cpad)            # logical position ids
+    tiles = idx.reshape(rpad // 128, 128, cpad // 4, 4).transpose(0, 2, 1, 3)
+    inter = tiles.reshape(rpad // 128, cpad // 4, 4, 32, 4).transpose(0, 1, 3, 2, 4)
+    stored = inter.reshape(-1)                                   # stored[byte] = logical id
+    pos = np.empty_like(stored)
+    pos[stored] = np.arange(stored.size)
+    return pos.reshape(rpad, cpad)
+
+
+def test_sf_layout_matches_documented_interleave():
+    for rows, K in [(1, 64), (128, 64), (130, 256), (300, 1344), (64, 16)]:
+        pos = _documented_sf_positions(rows, K)
+        got = np.array([[oracle.sf_offset(r, c, K) for c in range(pos.shape[1])] for r in range(pos.shape[0])])
+        assert np.array_equal(got, pos), (rows, K)
+    # the documented example: row 33, block 2 sits in the second 16-byte group
+    # at the second 4-byte slot
+    assert oracle.sf_offset(33, 2, 64) == 1 * 16 + 1 * 4 + 2
+
+
 def test_swizzle_roundtrip():
     rng = np.random.default_rng(9)
     for rows, K in [(200, 320), (64, 256), (5, 16)]:
@@ -388,6 +418,20 @@ def test_double_to_bf16_matches_torch_on_fp32_values():
     want = wl.bf16_bits(torch.from_numpy(v).to(torch.bfloat16))
     got = np.array([oracle.double_to_bf16(float(x)) for x in v], dtype=np.uint16)
     assert np.array_equal(got, want)
+
+
+def test_double_to_bf16_ties_go_to_even():
+    """fp32 values exactly halfway between two bf16 neighbours (low 16 bits
+    0x8000), over every exponent, both signs and both parities of the bf16
+    mantissa's last bit, subnormals included: round to the even neighbour,
+    as torch's fp32 -> bf16 conversion does."""
+    hi = np.arange(0, 0x7F7F, dtype=np.uint32)                   # every finite bf16 magnitude below the top
+    bits = np.concatenate([hi, hi | 0x8000]) << 16 | 0x8000
+    v = bits.astype(np.uint32).view(np.float32)
+    want = wl.bf16_bits(torch.from_numpy(v.copy()).to(torch.bfloat16))
+    got = np.array([oracle.double_to_bf16(float(x)) for x in v], dtype=np.uint16)
+    assert np.array_equal(got, want)
+    assert np.all((got & 1) == 0)                                # the even neighbour every time
 
 
 def test_swiglu_against_torch_float64():
