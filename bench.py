@@ -87,6 +87,11 @@ def parse_args():
     ap.add_argument("--no-side", action="store_true",
                     help="skip the side measurements (quantize, FP8 KV cache, decode) after the timed steps")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--side-only", choices=["quantize", "fp8_kv", "decode"], default=None,
+                    help="run only this side measurement (one GPU) and print it as one JSON line; "
+                         "for profiling the kernels behind it")
+    ap.add_argument("--decode-tokens", default="1,16,64,128",
+                    help="comma-separated tokens per decode step for the decode measurement")
     return ap.parse_args()
 
 
@@ -352,7 +357,7 @@ def bench_gpu(args, rank, world, local):
     if not args.no_side:
         quant = quantize_roofline(stack, pk, pk_kind)
         kv = fp8_kv_roofline(pk, pk_kind)
-        decode = decode_roofline(stack, pk, pk_kind)
+        decode = decode_roofline(stack, pk, pk_kind, decode_tokens(args))
 
     e2e = None
     if not args.no_e2e:
@@ -552,7 +557,9 @@ def decode_roofline(stack, pk, pk_kind, token_counts=(1, 16, 64, 128)):
                             outs[lin.N] = torch.empty((M, lin.N), dtype=torch.bfloat16, device=dev)
                         ops.linear_fused(src, qw, out=outs[lin.N], ws=ws)
 
+        l0 = ops.launch_count()
         step()
+        launches = ops.launch_count() - l0
         torch.cuda.synchronize()
         if ops.get_status() != 0:
             raise RuntimeError("device status set by the decode step")
@@ -577,7 +584,8 @@ def decode_roofline(stack, pk, pk_kind, token_counts=(1, 16, 64, 128)):
         ms = statistics.median(ts)
         gbs = wbytes / (ms * 1e-3) / 1e9
         res["steps"][str(M)] = {"us_per_step": round(ms * 1e3, 1), "us_per_linear": round(ms * 1e3 / 256, 2),
-                                "achieved": round(gbs, 1), "frac": round(gbs / pk["hbm_gbs"], 4)}
+                                "achieved": round(gbs, 1), "frac": round(gbs / pk["hbm_gbs"], 4),
+                                "gpu_launches_per_step": launches}
     return res
 
 
@@ -678,8 +686,33 @@ def bench_reference(args, rank, world):
     }
 
 
+def decode_tokens(args):
+    return tuple(int(t) for t in args.decode_tokens.split(","))
+
+
+def side_only(args):
+    """One side measurement on its own (one GPU), for profiling."""
+    from nvfp4_w4a4_quantized_act_b200 import build as nbuild
+    from nvfp4_w4a4_quantized_act_b200 import ops
+    nbuild.build()
+    if not ops.device_supported():
+        raise RuntimeError("the current device is not an sm_100 GPU")
+    pk, pk_kind = peaks()
+    if args.side_only == "fp8_kv":
+        return {"side": "fp8_kv", **fp8_kv_roofline(pk, pk_kind)}
+    stack = Stack(args.layers, "cuda:0")
+    if args.side_only == "quantize":
+        return {"side": "quantize", **quantize_roofline(stack, pk, pk_kind)}
+    return {"side": "decode", **decode_roofline(stack, pk, pk_kind, decode_tokens(args))}
+
+
 def main():
     args = parse_args()
+    if args.side_only is not None:
+        if int(os.environ.get("WORLD_SIZE", "1")) != 1:
+            raise SystemExit("--side-only runs on one GPU, without torchrun")
+        print(json.dumps(side_only(args)), flush=True)
+        return
     if args.impl == "reference":
         # the oracle arm runs on rank 0's host cores only; other ranks exit at once
         rank = int(os.environ.get("RANK", "0"))
