@@ -159,3 +159,73 @@ def test_fp8_kv_argument_errors_return_before_launch(L):
     assert L.nvfp4_fp8_kv_quantize(fake, 4, 16, 16, fake, fake, 20, None) == 3
     # empty tensors are no-ops
     assert L.nvfp4_fp8_kv_quantize(None, 0, 16, 16, fake, None, 16, None) == 0
+
+
+def test_segment_tables_are_checked_before_launch(L):
+    """Segments must be ordered, contiguous and cover [0, N); nseg in
+    [1, 16]; the table must exist.  Every case fails before any launch."""
+    fake = ctypes.c_void_p(1 << 20)
+    cases = {
+        "unsorted": [(10, 32), (0, 10)],
+        "overlapping": [(0, 20), (10, 32)],
+        "gap": [(0, 10), (12, 32)],
+        "past N": [(0, 10), (10, 40)],
+        "reversed": [(0, 20), (20, 10), (10, 32)],
+    }
+    for name, pairs in cases.items():
+        segs = _segarr(pairs)
+        assert L.nvfp4_gemm_prequant(fake, fake, fake, 8, 128, fake, fake, 32, segs, fake, len(pairs), fake, 0,
+                                     None) == 1, name
+        assert L.nvfp4_linear_fused(fake, 8, 128, fake, fake, 32, segs, fake, len(pairs), fake, 0, fake,
+                                    1 << 24, None) == 1, name
+        assert L.nvfp4_linear_fused_noalloc(fake, 8, 128, fake, fake, 32, segs, fake, len(pairs), fake, 0,
+                                            None) == 1, name
+    ok = _segarr([(0, 32)])
+    assert L.nvfp4_gemm_prequant(fake, fake, fake, 8, 128, fake, fake, 32, ok, fake, 0, fake, 0, None) == 1
+    assert L.nvfp4_gemm_prequant(fake, fake, fake, 8, 128, fake, fake, 32, None, fake, 1, fake, 0, None) == 1
+    assert L.nvfp4_quantize_weights(fake, 32, 64, 64, None, 1, fake, fake, fake, fake, 256, None) == 1
+
+
+def test_noalloc_limits_and_flags(L):
+    fake = ctypes.c_void_p(1 << 20)
+    one = _segarr([(0, 256)])
+    # the calibrated activation scale is not supported without a workspace
+    assert L.nvfp4_linear_fused_noalloc(fake, 8, 128, fake, fake, 256, one, fake, 1, fake, 1, None) == 1
+    # M * K above the fixed scratch
+    assert L.nvfp4_linear_fused_noalloc(fake, 1024, 8192, fake, fake, 256, one, fake, 1, fake, 0, None) == 7
+    # K % 64
+    assert L.nvfp4_linear_fused_noalloc(fake, 8, 96, fake, fake, 256, one, fake, 1, fake, 0, None) == 2
+
+
+def test_gated_entry_points_check_arguments_before_launch(L):
+    fake = ctypes.c_void_p(1 << 20)
+    mis = ctypes.c_void_p((1 << 20) + 8)
+    qws = ops.quant_workspace_bytes(2)
+    # gated weight quantize: F % 128, K % 16, ldw < K, misaligned ldw, workspace, null input
+    assert L.nvfp4_quantize_weights_gated(fake, 100, 64, 64, fake, fake, fake, fake, qws, None) == 2
+    assert L.nvfp4_quantize_weights_gated(fake, 128, 40, 40, fake, fake, fake, fake, qws, None) == 2
+    assert L.nvfp4_quantize_weights_gated(fake, 128, 64, 32, fake, fake, fake, fake, qws, None) == 1
+    assert L.nvfp4_quantize_weights_gated(fake, 128, 64, 68, fake, fake, fake, fake, qws, None) == 3
+    assert L.nvfp4_quantize_weights_gated(fake, 128, 64, 64, fake, fake, fake, fake, 4, None) == 7
+    assert L.nvfp4_quantize_weights_gated(None, 128, 64, 64, fake, fake, fake, fake, qws, None) == 1
+    # gated GEMM on quantized activations: F % 128, K % 64, workspace, misaligned h
+    assert L.nvfp4_gemm_prequant_swiglu(fake, fake, fake, 8, 128, fake, fake, 100, fake, fake, fake, 256,
+                                        None) == 2
+    assert L.nvfp4_gemm_prequant_swiglu(fake, fake, fake, 8, 96, fake, fake, 128, fake, fake, fake, 256,
+                                        None) == 2
+    assert L.nvfp4_gemm_prequant_swiglu(fake, fake, fake, 8, 128, fake, fake, 128, fake, fake, fake, 16,
+                                        None) == 7
+    assert L.nvfp4_gemm_prequant_swiglu(fake, fake, fake, 8, 128, fake, fake, 128, fake, mis, fake, 256,
+                                        None) == 3
+    # linear with the SwiGLU epilogue: unknown flag, F % 128, null g_h, misaligned h_codes, workspace
+    need = ops.workspace_bytes(8, 256, 128, 2)
+    assert L.nvfp4_linear_swiglu(fake, 8, 128, fake, fake, 128, fake, fake, fake, fake, fake, 1 << 12, fake,
+                                 need, None) == 1
+    assert L.nvfp4_linear_swiglu(fake, 8, 128, fake, fake, 96, fake, fake, fake, fake, fake, 0, fake, need,
+                                 None) == 2
+    assert L.nvfp4_linear_swiglu(fake, 8, 128, fake, fake, 128, fake, fake, fake, fake, None, 0, fake, need,
+                                 None) == 1
+    assert L.nvfp4_linear_swiglu(fake, 8, 128, fake, fake, 128, fake, fake, mis, fake, fake, 0, fake, need,
+                                 None) == 3
+    assert L.nvfp4_linear_swiglu(fake, 8, 128, fake, fake, 128, fake, fake, fake, fake, fake, 0, fake, need - 1,
+                                 None) == 7
