@@ -655,12 +655,31 @@ def oracle_sample_time(seconds: float, seed: int = 0):
             return flops, el, outs
 
 
+def oracle_codec_time():
+    """Time the oracle's activation codec on the whole activation-quantize
+    workload (X [8192, 5120], Student-t(3) with 1% of channels x100): amax,
+    global scale, block scales and codes.  Returns (elements, seconds)."""
+    import oracle
+    from nvfp4_w4a4_quantized_act_b200 import workloads as wl
+    xb = wl.bf16_bits(wl.act_quant_input())
+    t0 = time.perf_counter()
+    oracle.quantize_tensor(xb)
+    return xb.size, time.perf_counter() - t0
+
+
 def cpu_baseline(seconds: float):
     flops, el, outs = oracle_sample_time(seconds)
+    n_codec, t_codec = oracle_codec_time()
+    gate_up_flops = 2.0 * TOKENS * 2 * 17408 * HIDDEN
     return {"value": flops / el / 1e12, "unit": "TFLOPS", "cores": 1, "kind": "oracle",
             "sample": f"{outs} outputs of a [8192,5120]x[34816,5120]^T gate_up GEMM (K=5120) with on-the-fly "
                       f"quantization of the 64 activation rows and 256 weight rows they use, repeated for "
-                      f"{el:.1f} s; single-threaded C oracle, fp64 dot products"}
+                      f"{el:.1f} s; single-threaded C oracle, fp64 dot products",
+            "fp64_mac_per_s_with_quantization": round(flops / 2 / el, 1),
+            "gate_up_full_s_extrapolated": round(gate_up_flops / (flops / el), 1),
+            "codec": {"gbs": round(n_codec * (2 + 0.5 + 1 / 16) / t_codec / 1e9, 5), "seconds": round(t_codec, 2),
+                      "sample": "the whole [8192,5120] activation, dynamic scale (amax + block quantize), "
+                                "single-threaded; algorithmic bytes 2.5625 per element"}}
 
 
 def bench_reference(args, rank, world):
