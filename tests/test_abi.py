@@ -229,3 +229,45 @@ def test_gated_entry_points_check_arguments_before_launch(L):
                                  None) == 3
     assert L.nvfp4_linear_swiglu(fake, 8, 128, fake, fake, 128, fake, fake, fake, fake, fake, 0, fake, need - 1,
                                  None) == 7
+
+
+def _prototypes():
+    """name -> (return type, [parameter types]) for every function in the
+    header, comments removed, parameter names dropped."""
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    text = "\n".join(l for l in text.splitlines() if not l.lstrip().startswith("#"))
+    text = re.sub(r'extern\s+"C"\s*\{|\}', ";", text)
+    out = {}
+    for stmt in text.split(";"):
+        m = re.fullmatch(r"\s*([A-Za-z_][\w\s\*]*?)\b(nvfp4_[a-z0-9_]+)\s*\(([^)]*)\)\s*", stmt, flags=re.S)
+        if not m or stmt.lstrip().startswith("typedef"):
+            continue
+        ret, name, params = m.groups()
+        ps = [p.strip() for p in params.split(",") if p.strip() and p.strip() != "void"]
+        types = [re.sub(r"\b[A-Za-z_]\w*$", "", p).strip() if not p.endswith("*") else p for p in ps]
+        out[name] = (" ".join(ret.split()), [" ".join(t.split()) for t in types])
+    return out
+
+
+def _ctype_of(c_type):
+    if "nvfp4_segment" in c_type and "*" in c_type:
+        return ctypes.POINTER(ops.Segment)
+    if c_type.replace(" ", "") in ("constchar*", "char*"):
+        return ctypes.c_char_p
+    if "*" in c_type:
+        return ctypes.c_void_p
+    return {"int": ctypes.c_int, "unsigned": ctypes.c_uint, "int64_t": ctypes.c_int64, "size_t": ctypes.c_size_t,
+            "uint64_t": ctypes.c_uint64}[c_type.replace("const ", "")]
+
+
+def test_binding_signatures_match_the_header(L):
+    """Every ctypes restype/argtypes equals the header prototype's types
+    (pointer, segment table, 32/64-bit integer, size): a mismatch would pass
+    garbage silently."""
+    protos = _prototypes()
+    assert sorted(protos) == sorted(ops.EXPORTED)
+    for name, (ret, params) in protos.items():
+        f = getattr(L, name)
+        assert f.restype == _ctype_of(ret), (name, ret, f.restype)
+        assert list(f.argtypes) == [_ctype_of(p) for p in params], (name, params, f.argtypes)
