@@ -47,7 +47,7 @@ WORKLOAD = "496-linear hybrid stack (48 GDN + 16 attention layers, hidden 5120, 
 FP4_PER_BF16 = 4.0  # dense FP4 : dense BF16 tensor throughput on B200 (9 : 2.25 PFLOP/s nominal)
 FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # DRAM bytes (read + write) per GEMM launch, mean over the four GEMM launches of
-# one layer, from one ncu capture of this kernel source (profiles/
+# one layer, from one ncu capture of the GEMM sources with this code hash (profiles/
 # gemm_nvf4_pair_kernel_layer_8192tok.md gives the command: the DRAM-bytes
 # capture).  Reported only
 # while the kernel sources still have the captured hash.

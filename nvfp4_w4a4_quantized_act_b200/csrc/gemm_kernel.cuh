@@ -288,8 +288,10 @@ __device__ __forceinline__ void store_bf16_packed_128(const Params &p, int32_t r
         for (int j = 0; j < 64; j += 4)
             *reinterpret_cast<uint4 *>(o + 2 * j) = make_uint4(pk[j], pk[j + 1], pk[j + 2], pk[j + 3]);
     } else {
-        for (int j = 0; j < 128 && col0 + j < p.N; ++j)
-            o[j] = __ushort_as_bfloat16(static_cast<unsigned short>((j & 1) ? (pk[j >> 1] >> 16) : (pk[j >> 1] & 0xFFFFu)));
+#pragma unroll
+        for (int j = 0; j < 128; ++j)
+            if (col0 + j < p.N)
+                o[j] = __ushort_as_bfloat16(static_cast<unsigned short>((j & 1) ? (pk[j >> 1] >> 16) : (pk[j >> 1] & 0xFFFFu)));
     }
 }
 
@@ -551,10 +553,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                     for (int j = 0; j < 32; ++j)
                         hmax = vmax_mag(hmax, pk[j]);
                 } else {
-                    for (int j = 0; j < nval; ++j) {
-                        const uint32_t hb = (j & 1) ? (pk[j >> 1] >> 16) : (pk[j >> 1] & 0xFFFFu);
-                        o[j] = __ushort_as_bfloat16(static_cast<unsigned short>(hb));
-                        hmax = vmax_mag(hmax, hb);
+#pragma unroll
+                    for (int j = 0; j < 64; ++j) {
+                        if (j < nval) {
+                            const uint32_t hb = (j & 1) ? (pk[j >> 1] >> 16) : (pk[j >> 1] & 0xFFFFu);
+                            o[j] = __ushort_as_bfloat16(static_cast<unsigned short>(hb));
+                            hmax = vmax_mag(hmax, hb);
+                        }
                     }
                 }
             }

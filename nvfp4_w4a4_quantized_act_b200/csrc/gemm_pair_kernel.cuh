@@ -422,6 +422,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                 __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(p.out) + static_cast<int64_t>(row) * p.F + col0;
                 const int nval = min(64, p.F - col0);
                 if (p.tma_out) {
+#pragma unroll
                     for (int j = 0; j < 32; ++j) {
                         if (2 * j < nval)
                             hmax = vmax_mag(hmax, (2 * j + 1 < nval) ? pk[j] : (pk[j] & 0xFFFFu));
@@ -434,10 +435,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
                     for (int j = 0; j < 32; ++j)
                         hmax = vmax_mag(hmax, pk[j]);
                 } else {
-                    for (int j = 0; j < nval; ++j) {
-                        const uint32_t hb = (j & 1) ? (pk[j >> 1] >> 16) : (pk[j >> 1] & 0xFFFFu);
-                        o[j] = __ushort_as_bfloat16(static_cast<unsigned short>(hb));
-                        hmax = vmax_mag(hmax, hb);
+#pragma unroll
+                    for (int j = 0; j < 64; ++j) {
+                        if (j < nval) {
+                            const uint32_t hb = (j & 1) ? (pk[j >> 1] >> 16) : (pk[j >> 1] & 0xFFFFu);
+                            o[j] = __ushort_as_bfloat16(static_cast<unsigned short>(hb));
+                            hmax = vmax_mag(hmax, hb);
+                        }
                     }
                 }
             }

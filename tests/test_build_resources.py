@@ -18,9 +18,9 @@ from nvfp4_w4a4_quantized_act_b200 import build as nbuild
 
 # kernel (demangled-name fragment) -> (max registers, max stack bytes, max spill-store bytes)
 BUDGET = {
-    "gemm_nvf4_pair_kernel<true>": (128, 160, 16),
-    "gemm_nvf4_pair_kernel<false>": (128, 256, 16),
-    "gemm_nvf4_kernel<true>": (168, 128, 0),
+    "gemm_nvf4_pair_kernel<true>": (128, 0, 0),
+    "gemm_nvf4_pair_kernel<false>": (128, 16, 16),
+    "gemm_nvf4_kernel<true>": (168, 0, 0),
     "gemm_nvf4_kernel<false>": (168, 0, 0),
     "splitk_finalize_kernel": (255, 0, 0),
     "quantize_kernel": (64, 0, 0),
