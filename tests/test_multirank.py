@@ -49,3 +49,20 @@ def test_replicas_take_max_time_and_sum_work():
         assert elapsed == 20.0
         # 2 ranks x 1 TFLOP in 20 ms per step -> 100 TFLOPS
         assert abs(value - 100.0) < 1e-9
+
+
+def test_gemm_source_hash_ignores_comments_only(tmp_path, monkeypatch):
+    """The captured DRAM traffic is reported only while the GEMM sources
+    hash as captured: comment and whitespace edits keep the hash, any code
+    edit changes it."""
+    import bench
+    src = tmp_path / "k.cuh"
+    src.write_text("// a kernel\n__global__ void k(int *p) { p[0] = 1; /* store */ }\n")
+    monkeypatch.setattr(bench, "GEMM_SOURCES", [str(src)])
+    h0 = bench.gemm_source_hash()
+    src.write_text("// the kernel, reworded\n__global__   void k(int *p)\n{ p[0] = 1; /* one store */ }\n")
+    assert bench.gemm_source_hash() == h0
+    src.write_text("// a kernel\n__global__ void k(int *p) { p[0] = 2; /* store */ }\n")
+    assert bench.gemm_source_hash() != h0
+    monkeypatch.setattr(bench, "GEMM_TRAFFIC", {"source_sha256_12": h0, "bytes_per_launch": 1.0})
+    assert bench.gemm_traffic() is None
