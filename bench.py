@@ -47,13 +47,13 @@ WORKLOAD = "496-linear hybrid stack (48 GDN + 16 attention layers, hidden 5120, 
 FP4_PER_BF16 = 4.0  # dense FP4 : dense BF16 tensor throughput on B200 (9 : 2.25 PFLOP/s nominal)
 FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # DRAM bytes (read + write) per GEMM launch, mean over the four GEMM launches of
-# one layer, from one ncu capture of the GEMM sources with this code hash (profiles/
-# gemm_nvf4_pair_kernel_layer_8192tok.md gives the command: the DRAM-bytes
-# capture).  Reported only
-# while the kernel sources still have the captured hash.
+# one layer, from one ncu capture (the DRAM-bytes capture of these sources).
+# Reported only while the GEMM kernel sources and the host code that sets up
+# their launches (tile order, grid, tensor-map boxes, split-K) still hash to
+# the captured value.
 GEMM_TRAFFIC = {"source_sha256_12": "042d4e364773", "bytes_per_launch": 318.227e6}
 GEMM_SOURCES = [os.path.join(ROOT, "nvfp4_w4a4_quantized_act_b200", "csrc", f)
-                for f in ("gemm_kernel.cuh", "gemm_pair_kernel.cuh", "ptx_sm100.cuh")]
+                for f in ("gemm_kernel.cuh", "gemm_pair_kernel.cuh", "ptx_sm100.cuh", "nvfp4_api.cu")]
 
 
 def gemm_source_hash():
@@ -321,30 +321,39 @@ def bench_gpu(args, rank, world, local):
     if ops.get_status() != 0:
         raise RuntimeError("device status set during warm-up")
 
-    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_gemm)]
-          for _ in range(args.steps)]
     clocks = ClockSampler(local)
     l0 = ops.launch_count()
     barrier(world)
     torch.cuda.synchronize()
     clocks.start()
     time.sleep(0.3)
+    # the timed region: the steps alone, no event between kernels
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     t_start.record(stream)
     for s in range(args.steps):
-        stack.step_split(ev[s])
+        stack.step_split()
     t_end.record(stream)
     torch.cuda.synchronize()
     barrier(world)
     clk = clocks.stop()
     launches = ops.launch_count() - l0
     elapsed_ms = max_over_ranks(t_start.elapsed_time(t_end), world)
-    gemm_ms = [sum(ev[s][k][0].elapsed_time(ev[s][k][1]) for s in range(args.steps)) / args.steps
-               for k in range(n_gemm)]
     status = ops.get_status()
     if status != 0:
         raise RuntimeError(f"device status {status} after the timed region")
+    # a separate, untimed pass of the same steps with CUDA events around each
+    # GEMM launch: the GEMM kernel's own durations for the roofline
+    gemm_steps = max(2, min(args.steps, 5))
+    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_gemm)]
+          for _ in range(gemm_steps)]
+    for s in range(gemm_steps):
+        stack.step_split(ev[s])
+    torch.cuda.synchronize()
+    gemm_ms = [sum(ev[s][k][0].elapsed_time(ev[s][k][1]) for s in range(gemm_steps)) / gemm_steps
+               for k in range(n_gemm)]
+    if ops.get_status() != 0:
+        raise RuntimeError("device status set during the GEMM-duration pass")
 
     ms_per_step = elapsed_ms / args.steps
     value = aggregate_throughput(stack.flops, world, ms_per_step)
@@ -403,6 +412,9 @@ def bench_gpu(args, rank, world, local):
         "fp8_kv_roofline": kv,
         "decode_roofline": decode,
         "gemm_share_of_step": round(sum(gemm_ms) / ms_per_step, 4),
+        "timing": {"ms_per_step": "CUDA events around the K timed steps only, no event between kernels",
+                   "gemm": f"roofline.achieved and gemm_share_of_step from a separate untimed pass of "
+                           f"{gemm_steps} steps with CUDA events around each of the {n_gemm} GEMM launches"},
         "gpu_launches": int(launches),
         "clocks": clk,
     }
@@ -626,19 +638,25 @@ def bench_e2e(stack, args, world):
 
 # ------------------------------------------------------ CPU oracle legs
 
-def oracle_sample_time(seconds: float, seed: int = 0):
+def oracle_sample_operands():
+    """bf16 bits of the 64 activation rows and 256 gate_up weight rows the
+    oracle sample draws its outputs from."""
+    from nvfp4_w4a4_quantized_act_b200 import workloads as wl
+    x = wl.activation_normal(64, HIDDEN, 11)
+    w = wl.weight_normal(256, HIDDEN, 0.02, 1000)
+    return wl.bf16_bits(x), wl.bf16_bits(w)
+
+
+def oracle_sample_time(seconds: float, seed: int = 0, operands=None):
     """Time the oracle on a bounded sample of the stack: quantize the rows it
     needs of one activation and one gate_up weight, then compute sampled
     outputs of that GEMM by fp64 dot products, until `seconds` pass.
     Returns (flops, seconds, outputs)."""
     import oracle
-    from nvfp4_w4a4_quantized_act_b200 import workloads as wl
     rng = np.random.default_rng(seed)
     K = HIDDEN
     rows = 64
-    x = wl.activation_normal(rows, K, 11)
-    w = wl.weight_normal(256, K, 0.02, 1000)
-    xb, wb = wl.bf16_bits(x), wl.bf16_bits(w)
+    xb, wb = operands if operands is not None else oracle_sample_operands()
     flops = 0.0
     outs = 0
     t0 = time.perf_counter()
@@ -661,46 +679,146 @@ def oracle_codec_time():
     global scale, block scales and codes.  Returns (elements, seconds)."""
     import oracle
     from nvfp4_w4a4_quantized_act_b200 import workloads as wl
-    xb = wl.bf16_bits(wl.act_quant_input())
+    xb = _CODEC_X if _CODEC_X is not None else wl.bf16_bits(wl.act_quant_input())
     t0 = time.perf_counter()
     oracle.quantize_tensor(xb)
     return xb.size, time.perf_counter() - t0
 
 
-def cpu_baseline(seconds: float):
-    flops, el, outs = oracle_sample_time(seconds)
-    n_codec, t_codec = oracle_codec_time()
+def host_cores() -> int:
+    """Cores this process may run on (the container's share of the host)."""
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:  # pragma: no cover
+        return os.cpu_count() or 1
+
+
+def host_cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+# The activation the parallel codec timing quantizes, made before the worker
+# pool is forked so that every worker reads the parent's copy.
+_CODEC_X = None
+_SAMPLE_OPERANDS = None
+
+
+def _pool_gemm_sample(args):
+    seconds, seed = args
+    return oracle_sample_time(seconds, seed, _SAMPLE_OPERANDS)
+
+
+def _pool_codec_amax(rows):
+    import oracle
+    return oracle.amax(_CODEC_X, rows[0], rows[1])
+
+
+def _pool_codec_quantize(args):
+    import oracle
+    r0, r1, g = args
+    codes, scales = oracle.quantize(np.ascontiguousarray(_CODEC_X[r0:r1]), g)
+    return int(codes[:, :1].sum()) + int(scales[:, :1].sum())
+
+
+class OraclePool:
+    """One worker process per host core running the oracle, unchanged, on
+    disjoint pieces of the work: sampled GEMM outputs (each worker its own
+    seed) and the rows of the activation codec (amax of each worker's rows,
+    their maximum, then each worker quantizes its rows with the global
+    scale).  The pool is forked before any CUDA call of this process (a fork
+    after one is unsafe); workers never touch the GPU."""
+
+    def __init__(self, cores: int | None = None):
+        global _CODEC_X, _SAMPLE_OPERANDS
+        import multiprocessing as mp
+        from nvfp4_w4a4_quantized_act_b200 import workloads as wl
+        import oracle
+        oracle.build()
+        self.cores = cores or host_cores()
+        # inputs made here, before the fork: the workers use no torch
+        _CODEC_X = wl.bf16_bits(wl.act_quant_input())
+        _SAMPLE_OPERANDS = oracle_sample_operands()
+        self.pool = mp.get_context("fork").Pool(self.cores)
+
+    def gemm_rate(self, seconds: float, seed0: int = 100):
+        """(flops, seconds, outputs) of all workers together: the work of
+        every worker over the longest worker's time."""
+        res = self.pool.map(_pool_gemm_sample, [(seconds, seed0 + i) for i in range(self.cores)])
+        return sum(r[0] for r in res), max(r[1] for r in res), sum(r[2] for r in res)
+
+    def codec_time(self):
+        import oracle
+        rows = _CODEC_X.shape[0]
+        cuts = np.linspace(0, rows, self.cores + 1).astype(int)
+        parts = [(int(a), int(b)) for a, b in zip(cuts[:-1], cuts[1:]) if b > a]
+        t0 = time.perf_counter()
+        a = max(self.pool.map(_pool_codec_amax, parts))
+        g = oracle.global_scale(a)
+        self.pool.map(_pool_codec_quantize, [(r0, r1, g) for r0, r1 in parts])
+        return _CODEC_X.size, time.perf_counter() - t0
+
+    def close(self):
+        self.pool.terminate()
+        self.pool.join()
+
+
+def cpu_baseline(seconds: float, pool: OraclePool):
+    """The oracle on the host cores: all of them (the baseline's value) and
+    one (for reference)."""
     gate_up_flops = 2.0 * TOKENS * 2 * 17408 * HIDDEN
-    return {"value": flops / el / 1e12, "unit": "TFLOPS", "cores": 1, "kind": "oracle",
-            "sample": f"{outs} outputs of a [8192,5120]x[34816,5120]^T gate_up GEMM (K=5120) with on-the-fly "
-                      f"quantization of the 64 activation rows and 256 weight rows they use, repeated for "
-                      f"{el:.1f} s; single-threaded C oracle, fp64 dot products",
-            "fp64_mac_per_s_with_quantization": round(flops / 2 / el, 1),
-            "gate_up_full_s_extrapolated": round(gate_up_flops / (flops / el), 1),
-            "codec": {"gbs": round(n_codec * (2 + 0.5 + 1 / 16) / t_codec / 1e9, 5), "seconds": round(t_codec, 2),
-                      "sample": "the whole [8192,5120] activation, dynamic scale (amax + block quantize), "
-                                "single-threaded; algorithmic bytes 2.5625 per element"}}
+    f1, el1, outs1 = oracle_sample_time(seconds)
+    n_codec, t_codec1 = oracle_codec_time()
+    fa, ela, outsa = pool.gemm_rate(seconds)
+    _, t_codeca = pool.codec_time()
+    codec_bytes = n_codec * (2 + 0.5 + 1 / 16)
+    return {"value": fa / ela / 1e12, "unit": "TFLOPS", "cores": pool.cores, "kind": "oracle",
+            "cores_host": host_cores(), "cpu_model": host_cpu_model(),
+            "value_all_cores": fa / ela / 1e12, "value_1core": f1 / el1 / 1e12,
+            "sample": f"sampled outputs of a [8192,5120]x[34816,5120]^T gate_up GEMM (K=5120) with on-the-fly "
+                      f"quantization of the 64 activation rows and 256 weight rows each batch uses, repeated "
+                      f"for {seconds:.0f} s: {outsa} outputs on {pool.cores} worker processes (one per core), "
+                      f"{outs1} on one core; C oracle, fp64 dot products",
+            "fp64_mac_per_s_with_quantization": {"all_cores": round(fa / 2 / ela, 1), "1core": round(f1 / 2 / el1, 1)},
+            "gate_up_full_s_extrapolated": {"all_cores": round(gate_up_flops / (fa / ela), 1),
+                                            "1core": round(gate_up_flops / (f1 / el1), 1)},
+            "codec": {"gbs": round(codec_bytes / t_codeca / 1e9, 5), "seconds": round(t_codeca, 2),
+                      "gbs_1core": round(codec_bytes / t_codec1 / 1e9, 5), "seconds_1core": round(t_codec1, 2),
+                      "sample": "the whole [8192,5120] activation, dynamic scale (amax + block quantize); "
+                                "rows split across the worker processes; algorithmic bytes 2.5625 per element"}}
 
 
 def bench_reference(args, rank, world):
     if rank != 0:
         return None
-    per_step = max(2.0, min(20.0, 60.0 / max(1, args.steps + args.warmup)))
-    for _ in range(args.warmup):
-        oracle_sample_time(per_step / 4)
-    tot_f, tot_t = 0.0, 0.0
-    for _ in range(args.steps):
-        f, t, outs = oracle_sample_time(per_step)
-        tot_f += f
-        tot_t += t
+    pool = OraclePool()
+    try:
+        per_step = max(2.0, min(20.0, 60.0 / max(1, args.steps + args.warmup)))
+        for _ in range(args.warmup):
+            pool.gemm_rate(per_step / 4)
+        tot_f, tot_t = 0.0, 0.0
+        for _ in range(args.steps):
+            f, t, outs = pool.gemm_rate(per_step)
+            tot_f += f
+            tot_t += t
+    finally:
+        pool.close()
     v = tot_f / tot_t / 1e12
     return {
         "impl": "reference", "metric": METRIC, "value": v, "unit": "TFLOPS", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": tot_t / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64 (oracle GEMM)",
         "data": "synthetic", "config": {"workload": WORKLOAD, "tokens": TOKENS, "hidden": HIDDEN},
-        "cpu_baseline": {"value": v, "unit": "TFLOPS", "cores": 1, "kind": "oracle",
-                         "sample": f"each step: {per_step:.1f} s of sampled gate_up outputs with quantization"},
+        "cpu_baseline": {"value": v, "unit": "TFLOPS", "cores": pool.cores, "kind": "oracle",
+                         "cores_host": host_cores(), "cpu_model": host_cpu_model(),
+                         "sample": f"each step: {per_step:.1f} s of sampled gate_up outputs with quantization "
+                                   f"on {pool.cores} worker processes (one per core)"},
         "e2e": {"value": v, "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 
@@ -739,14 +857,20 @@ def main():
         if res is not None:
             print(json.dumps(res), flush=True)
         return
+    # the oracle's worker pool is forked before this process makes any CUDA call
+    pool = None
+    if int(os.environ.get("RANK", "0")) == 0 and not args.no_cpu_baseline:
+        pool = OraclePool()
     rank, world, local = dist_setup(args)
     try:
         res = bench_gpu(args, rank, world, local)
-        if rank == 0 and res is not None and not args.no_cpu_baseline:
-            res["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
+        if rank == 0 and res is not None and pool is not None:
+            res["cpu_baseline"] = cpu_baseline(args.cpu_seconds, pool)
         if rank == 0 and res is not None:
             print(json.dumps(res), flush=True)
     finally:
+        if pool is not None:
+            pool.close()
         if world > 1:
             import torch.distributed as dist
             dist.destroy_process_group()

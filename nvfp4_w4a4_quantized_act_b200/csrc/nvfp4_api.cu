@@ -848,8 +848,9 @@ static_assert(kNoAllocSfOff % 1024 == 0, "scale factors must stay 16-byte aligne
 static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocBytes];
 
 // Device address of g_noalloc_scratch per device (the host-side symbol is a
-// stand-in, never a device pointer).
-uint8_t *g_noalloc_ptr[kMaxDevices] = {};
+// stand-in, never a device pointer).  Written once per device under the
+// mutex (release), read without it (acquire).
+std::atomic<uint8_t *> g_noalloc_ptr[kMaxDevices] = {};
 std::mutex g_noalloc_mu;
 
 uint8_t *noalloc_scratch()
@@ -857,16 +858,19 @@ uint8_t *noalloc_scratch()
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
         return nullptr;
-    if (g_noalloc_ptr[dev] != nullptr)
-        return g_noalloc_ptr[dev];
+    uint8_t *known = g_noalloc_ptr[dev].load(std::memory_order_acquire);
+    if (known != nullptr)
+        return known;
     std::lock_guard<std::mutex> lock(g_noalloc_mu);
-    if (g_noalloc_ptr[dev] == nullptr) {
+    known = g_noalloc_ptr[dev].load(std::memory_order_relaxed);
+    if (known == nullptr) {
         void *p = nullptr;
         if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
             return nullptr;
-        g_noalloc_ptr[dev] = static_cast<uint8_t *>(p);
+        known = static_cast<uint8_t *>(p);
+        g_noalloc_ptr[dev].store(known, std::memory_order_release);
     }
-    return g_noalloc_ptr[dev];
+    return known;
 }
 
 }  // namespace

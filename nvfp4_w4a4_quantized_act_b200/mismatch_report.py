@@ -41,7 +41,10 @@ def _rel_err(y: np.ndarray, ref: np.ndarray) -> float:
     return float(np.linalg.norm(y - ref) / max(np.linalg.norm(ref), 1e-300))
 
 
-def run(tokens: int = 16384, rows: int = 256, seed: int = 3) -> dict:
+def run(tokens: int = 16384, rows: int = 256, seed: int = 3, keep_outputs: bool = False) -> dict:
+    """Serve the fused weight the three ways; per module, the relative error
+    of each against X W^T.  keep_outputs adds the sampled fp32 outputs
+    ('outputs': name -> [rows, N]) and their token indices ('rows')."""
     lin = wl.gdn_inproj_linear(seed)
     segs = lin.segments
     K, N = lin.K, lin.N
@@ -75,8 +78,12 @@ def run(tokens: int = 16384, rows: int = 256, seed: int = 3) -> dict:
             "rel_err_mismatch": _rel_err(outs["mismatch"][:, a:b], ref[:, a:b]),
             "rel_err_shared": _rel_err(outs["shared"][:, a:b], ref[:, a:b]),
         })
-    return {"tokens": tokens, "K": K, "N": N, "rows_sampled": int(len(pick)), "g_shared": g_shared,
-            "status": status, "modules": modules}
+    res = {"tokens": tokens, "K": K, "N": N, "rows_sampled": int(len(pick)), "g_shared": g_shared,
+           "status": status, "modules": modules}
+    if keep_outputs:
+        res["outputs"] = outs
+        res["rows"] = pick
+    return res
 
 
 def main():

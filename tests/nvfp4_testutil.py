@@ -75,3 +75,63 @@ def sample_outputs(M: int, N: int, segments, rng: np.random.Generator, n_random:
             ms.append(r)
             ns.append(c)
     return np.array(ms, dtype=np.int64), np.array(ns, dtype=np.int64)
+
+
+def check_gemm_bf16(out_bits: np.ndarray, C: np.ndarray, B: np.ndarray, what: str = "") -> float:
+    """bf16 outputs: the fp32 tolerance plus half a bf16 ulp of the output."""
+    v = oracle.bf16_bits_to_f32(out_bits).astype(np.float64)
+    a = np.maximum(np.abs(v), 1e-38)
+    ulp = np.exp2(np.floor(np.log2(a)) - 7)
+    tol = oracle.gemm_tolerance(B) + 0.5 * ulp
+    err = np.abs(v - C)
+    bad = err > tol
+    assert not np.any(bad), f"{what}: {int(bad.sum())} outside tolerance, e.g. gpu={v[bad][:3]} oracle={C[bad][:3]}"
+    return float(np.max(err / tol)) if err.size else 0.0
+
+
+def oracle_sampled(xb, wb, segments, ms, ns):
+    """Oracle outputs at the sampled (m, n) pairs: the tensor-wide global
+    scales come from the whole operands, the codes and block scales only
+    from the rows the samples use."""
+    g_a = oracle.global_scale(oracle.amax(xb))
+    gseg = oracle.segment_scales(wb, segments)
+    grow = oracle.rows_scale(segments, gseg, wb.shape[0])
+    um, im = np.unique(ms, return_inverse=True)
+    un, inn = np.unique(ns, return_inverse=True)
+    ac, asc = oracle.quantize(np.ascontiguousarray(xb[um]), g_a)
+    wc, wsc = oracle.quantize(np.ascontiguousarray(wb[un]), grow[un])
+    C, B = oracle.linear_sampled(ac, asc, g_a, wc, wsc, grow[un], im, inn)
+    return C, B, (um, ac, asc, np.float32(g_a)), (un, wc, wsc, gseg)
+
+
+def full_size_check(X, W, segments, seed):
+    """nvfp4_linear_fused at full size (bf16 and fp32 outputs) against the
+    oracle on sampled outputs; the quantized operands of the sampled rows
+    are checked bit for bit.  Returns the largest error / tolerance ratio."""
+    M, K = X.shape
+    N = W.shape[0]
+    xb, wb = wl.bf16_bits(X), wl.bf16_bits(W)
+    qw = ops.quantize_weights(W.to(DEV), segments)
+    Xd = X.to(DEV)
+    ws = torch.empty(ops.workspace_bytes(M, N, K, len(segments)), dtype=torch.uint8, device=DEV)
+    out = ops.linear_fused(Xd, qw, ws=ws)
+    out32 = ops.linear_fused(Xd, qw, ws=ws, out_fp32=True)
+    assert ops.get_status() == 0
+    rng = np.random.default_rng(seed)
+    ms, ns = sample_outputs(M, N, segments, rng)
+    C, B, (um, ac, asc, ga), (un, wc, wsc, gseg) = oracle_sampled(xb, wb, segments, ms, ns)
+    # quantized operands of the sampled rows are the oracle's, bit for bit
+    g_ws, c_ws, sf_ws = ops.linear_workspace_views(ws, M, K)
+    assert float(host(g_ws)[0]) == float(ga)
+    assert np.array_equal(host(qw.g_w), gseg)
+    assert np.array_equal(host(c_ws)[um], ac)
+    assert np.array_equal(oracle.unswizzle(host(sf_ws), M, K)[um], asc)
+    assert np.array_equal(host(qw.codes)[un], wc)
+    sf_w = host(qw.sf)
+    assert np.array_equal(oracle.unswizzle(sf_w, N, K)[un], wsc)
+    o32 = host(out32)[ms, ns]
+    r32 = check_gemm(o32, C, B, "fp32 sampled")
+    o16 = host(out.view(torch.int16)).view(np.uint16)[ms, ns]
+    check_gemm_bf16(o16, C, B, "bf16 sampled")
+    assert np.array_equal(o16, bf16_of_f32(o32))
+    return r32

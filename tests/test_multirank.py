@@ -66,3 +66,14 @@ def test_gemm_source_hash_ignores_comments_only(tmp_path, monkeypatch):
     assert bench.gemm_source_hash() != h0
     monkeypatch.setattr(bench, "GEMM_TRAFFIC", {"source_sha256_12": h0, "bytes_per_launch": 1.0})
     assert bench.gemm_traffic() is None
+
+
+def test_gemm_source_hash_covers_the_launch_code():
+    """The hash also covers the host code that chooses the GEMM's tile
+    order, grid, tensor-map boxes and split-K (nvfp4_api.cu): a change
+    there invalidates the captured traffic too."""
+    import bench
+    names = [os.path.basename(p) for p in bench.GEMM_SOURCES]
+    assert "nvfp4_api.cu" in names
+    assert {"gemm_kernel.cuh", "gemm_pair_kernel.cuh", "ptx_sm100.cuh"} <= set(names)
+    assert all(os.path.exists(p) for p in bench.GEMM_SOURCES)

@@ -5,11 +5,13 @@ runs (a host runtime that owns all device memory and gives its operators no
 allocator, or a serving loop that must not pay cudaMalloc's device-wide
 synchronization).  Its scratch lives in a fixed device array inside the
 library, so these tests check that:
-  * two calls in a row through the C ABI give the same result as the
-    workspace-taking nvfp4_linear_fused on the same inputs, within the GEMM
-    tolerance the other tests use (and, since both run the same kernels,
-    bit for bit) -- the second call uses a tensor with a much smaller amax,
-    so a stale amax left in the shared scratch would show;
+  * two calls in a row through the C ABI agree with the oracle within the
+    GEMM tolerance the other tests use, and with the workspace-taking
+    nvfp4_linear_fused on the same inputs -- the second call uses a tensor
+    with a much smaller amax, so a stale amax left in the shared scratch
+    would show;
+  * decode-sized inputs (M <= 128, the single-CTA kernel without split-K)
+    agree with the oracle the same way, on a ragged N with several modules;
   * inputs larger than the array are refused before anything runs.
 This file is collected last on purpose: a failure here stops an -x run only
 after every other test has run.
@@ -38,7 +40,14 @@ def _call_noalloc(X, qw, out, flags=0):
         ctypes.c_void_p(out.data_ptr()), flags, ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
 
 
-def test_noalloc_matches_workspace_entry_point_twice():
+def _oracle_check(X, cw, sw, grow, got):
+    ca, sa, ga = oracle.quantize_tensor(wl.bf16_bits(X))
+    C, B = oracle.linear_full(ca, sa, ga, cw, sw, grow)
+    err = np.abs(got.cpu().numpy().astype(np.float64) - C)
+    assert np.all(err <= oracle.gemm_tolerance(B)), float(np.max(err / oracle.gemm_tolerance(B)))
+
+
+def test_noalloc_matches_oracle_and_workspace_entry_point_twice():
     widths = [96, 160, 48]
     segs = wl.segments_from_widths(widths)
     K = 1024
@@ -59,12 +68,31 @@ def test_noalloc_matches_workspace_entry_point_twice():
         assert _call_noalloc(Xd, qw, got16) == 0
         ref16 = ops.linear_fused(Xd, qw)
         assert ops.get_status() == 0
-        ca, sa, ga = oracle.quantize_tensor(wl.bf16_bits(X))
-        _, B = oracle.linear_full(ca, sa, ga, cw, sw, grow)
-        diff = np.abs(got.cpu().numpy().astype(np.float64) - ref.cpu().numpy().astype(np.float64))
-        assert np.all(diff <= oracle.gemm_tolerance(B))
+        _oracle_check(X, cw, sw, grow, got)
+        # both entry points run the same kernels on the same operands
         assert torch.equal(got, ref)
         assert torch.equal(got16, ref16)
+
+
+def test_noalloc_decode_sizes_match_oracle():
+    """M <= 128: the allocation-free call runs the single-CTA GEMM over the
+    whole K (it has no room for split-K partials), so it is compared with the
+    oracle, not bit for bit with nvfp4_linear_fused (which may split K)."""
+    widths = [200, 72, 48, 17]  # N = 337: a ragged last tile
+    segs = wl.segments_from_widths(widths)
+    K = 2048
+    W = torch.cat([wl.weight_normal(w, K, s, 80 + i)
+                   for i, (w, s) in enumerate(zip(widths, [0.02, 0.005, 0.05, 0.01]))])
+    qw = ops.quantize_weights(W.to(DEV), segs)
+    cw, sw, gseg = oracle.quantize_segments(wl.bf16_bits(W), segs)
+    grow = oracle.rows_scale(segs, gseg, W.shape[0])
+    for M, seed in ((1, 81), (16, 82), (100, 83), (16, 84)):
+        X = wl.activation_normal(M, K, seed, n_outliers=2 if seed % 2 else 0)
+        got = torch.full((M, qw.N), float("nan"), dtype=torch.float32, device=DEV)
+        rc = _call_noalloc(X.to(DEV), qw, got, ops.NVFP4_OUT_FP32)
+        assert rc == 0, ops.status_string(rc)
+        assert ops.get_status() == 0
+        _oracle_check(X, cw, sw, grow, got)
 
 
 def test_noalloc_rejects_oversize_and_static_scale():
