@@ -457,33 +457,77 @@ def _timed_flushed(fn, flush, reps=13, skip=3):
     return statistics.median(ts)
 
 
+def _timed_rotating(fn, n_inputs, rounds=4, reps=7, skip=2):
+    """Median time per call of fn(i), called for i = 0 .. n_inputs-1 `rounds`
+    times back to back between two CUDA events: with the inputs together
+    larger than L2, no call finds its own input there, and each call's launch
+    overlaps the previous one as it would inside a step."""
+    ts = []
+    for r in range(reps):
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        for _ in range(rounds):
+            for i in range(n_inputs):
+                fn(i)
+        e.record()
+        e.synchronize()
+        if r >= skip:
+            ts.append(s.elapsed_time(e) / (rounds * n_inputs))
+    return statistics.median(ts)
+
+
 def quantize_roofline(stack, pk, pk_kind):
-    """Activation quantization of X [8192, 5120] with L2 flushed: the dynamic
-    path (amax pass + quantize pass, the roofline figure) and the calibrated
-    single pass.  For context, the time of one read of X by a plain torch
-    reduction under the same flush (the read alone, no writes)."""
+    """Activation quantization of X [8192, 5120] (the stack's GDN/attention
+    input): the dynamic path (clearing + amax + quantize launches, the
+    roofline figure) and the calibrated single pass.  Timed as 16 calls back
+    to back over 4 distinct inputs and outputs (4 x 107.5 MB, more than the
+    126 MB L2), per call = total / 16.  For context: one call with L2 flushed
+    before it (launch latency included in its events), and one read of X by a
+    plain torch reduction under the same flush."""
     from nvfp4_w4a4_quantized_act_b200 import ops
+    from nvfp4_w4a4_quantized_act_b200 import workloads as wl
     X = stack.X
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=X.device)
-    ms = _timed_flushed(lambda: ops.quantize_act(X, g_a=stack.g_a, codes=stack.a_codes, sf=stack.a_sf,
-                                                 ws=stack.qws), flush)
-    ms_static = _timed_flushed(lambda: ops.quantize_act(X, g_a=stack.g_a, codes=stack.a_codes, sf=stack.a_sf,
-                                                        ws=stack.qws, static_scale=True), flush)
+    dev = X.device
+    n_in = 4
+    xs = [X] + [wl.activation_normal_cuda(TOKENS, HIDDEN, 21 + i, device=dev) for i in range(n_in - 1)]
+    bufs = [(torch.empty(TOKENS * HIDDEN // 2, dtype=torch.uint8, device=dev),
+             torch.empty(ops.sf_bytes(TOKENS, HIDDEN), dtype=torch.uint8, device=dev),
+             torch.empty(1, dtype=torch.float32, device=dev),
+             torch.empty(ops.quant_workspace_bytes(1), dtype=torch.uint8, device=dev)) for _ in range(n_in)]
+
+    def call(i, static):
+        c, sf, g, ws = bufs[i]
+        ops.quantize_act(xs[i], g_a=g, codes=c, sf=sf, ws=ws, static_scale=static)
+
+    for i in range(n_in):  # calibrated scales for the static pass: the inputs' own
+        call(i, False)
+    torch.cuda.synchronize()
+    ms = _timed_rotating(lambda i: call(i, False), n_in)
+    ms_static = _timed_rotating(lambda i: call(i, True), n_in)
+    if ops.get_status() != 0:
+        raise RuntimeError("device status set by the quantize measurement")
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    ms_one = _timed_flushed(lambda: call(0, False), flush)
+    ms_one_static = _timed_flushed(lambda: call(0, True), flush)
     xi = X.view(torch.int32)
     ms_read = _timed_flushed(lambda: xi.max(), flush)
+    del xs, bufs, flush
     alg = TOKENS * HIDDEN * (2 + 0.5 + 1 / 16)
     gbs = alg / (ms * 1e-3) / 1e9
-    return {"kernel": "amax_kernel + quantize_kernel (dynamic per-tensor scale), X [8192, 5120] bf16",
+    return {"kernel": "zero_words_kernel + amax_kernel + quantize_act_kernel (dynamic per-tensor scale), "
+                      "X [8192, 5120] bf16",
             "bound": "hbm", "achieved": round(gbs, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
             "frac": round(gbs / pk["hbm_gbs"], 4), "us": round(ms * 1e3, 2),
             "algorithmic_bytes": int(alg), "peak_basis": pk_kind,
-            "l2": "256 MB written and read back before each launch",
+            "l2": "16 calls back to back over 4 distinct inputs and outputs (4 x 107.5 MB > 126 MB L2)",
             "static_scale_us": round(ms_static * 1e3, 2),
             "static_scale_gbs": round(alg / (ms_static * 1e-3) / 1e9, 1),
+            "static_scale_frac": round(alg / (ms_static * 1e-3) / 1e9 / pk["hbm_gbs"], 4),
+            "one_call_l2_flushed_us": {"dynamic": round(ms_one * 1e3, 2), "static": round(ms_one_static * 1e3, 2),
+                                       "note": "256 MB written and read back before the call; its events "
+                                               "include the launch latency"},
             "torch_read_of_x_us": round(ms_read * 1e3, 2),
-            "torch_read_of_x_gbs": round(X.numel() * 2 / (ms_read * 1e-3) / 1e9, 1),
-            # the calibrated single pass's byte rate against a plain read of X of the same size
-            "static_frac_of_plain_read_rate": round((alg / ms_static) / (X.numel() * 2 / ms_read), 3)}
+            "torch_read_of_x_gbs": round(X.numel() * 2 / (ms_read * 1e-3) / 1e9, 1)}
 
 
 def fp8_kv_roofline(pk, pk_kind):

@@ -65,4 +65,30 @@ __device__ __forceinline__ void div_shared_x2(uint32_t w, float d, float nr, flo
         : "f"(nx_lo), "f"(nx_hi), "f"(d), "f"(nr));
 }
 
+// The negated quotients -(x/d) of the two bf16 values packed in w, computed
+// from x itself (no negation of the inputs): with nr = -RN(1/d),
+//     q = RN(x nr),  e = RN(d q + x),  -y = RN(e nr + q).
+// Each step is the exact negation of the matching div_shared step: rounding
+// to nearest is symmetric, and where a sum is exactly zero the two forms may
+// differ only in the sign of that zero, which reaches the result only for
+// x = +-0, where it gives the negated signed zero as well (x = -0 yields
+// +0 = -(-0)).  So the results are bit-identical to -div_shared(x, d, RN(1/d)).  The quantizer
+// encodes -y and flips the sign bit of every code afterwards, one XOR per
+// eight codes instead of one per two inputs.
+__device__ __forceinline__ void div_shared_neg_x2(uint32_t w, float d, float nr, float &n_lo, float &n_hi)
+{
+    asm("{\n\t.reg .b32 l, h;\n\t.reg .b64 x, q, e, dd, rr;\n\t"
+        "shl.b32 l, %2, 16;\n\t"
+        "and.b32 h, %2, 0xFFFF0000;\n\t"
+        "mov.b64 x, {l, h};\n\t"
+        "mov.b64 dd, {%3, %3};\n\t"
+        "mov.b64 rr, {%4, %4};\n\t"
+        "mul.rn.f32x2 q, x, rr;\n\t"     // q = RN(x nr) = -RN(x r)
+        "fma.rn.f32x2 e, dd, q, x;\n\t"  // e = RN(x - d RN(x r))
+        "fma.rn.f32x2 q, e, rr, q;\n\t"  // -y = RN(-(RN(x r) + e r))
+        "mov.b64 {%0, %1}, q;\n\t}"
+        : "=f"(n_lo), "=f"(n_hi)
+        : "r"(w), "f"(d), "f"(nr));
+}
+
 }  // namespace nvfp4

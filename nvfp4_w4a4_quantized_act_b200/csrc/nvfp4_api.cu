@@ -191,6 +191,17 @@ int run_amax(DeviceState *d, const void *X, int64_t rows, int64_t K, int64_t ld,
     return NVFP4_OK;
 }
 
+// The block quantizer: the single-segment kernel for activations (one global
+// scale, rows in order), the general one for module segments or the gated
+// row order.
+void launch_quantize(const nvfp4::QuantParams &p, int grid, cudaStream_t stream)
+{
+    if (p.seg.nseg == 1 && p.gate_up_F == 0)
+        launch(nvfp4::quantize_act_kernel, dim3(grid), dim3(256), 0, stream, p);
+    else
+        launch(nvfp4::quantize_kernel, dim3(grid), dim3(256), 0, stream, p);
+}
+
 // K1 + K2 for `rows` x K bf16 rows, segment table `seg`.  mode 0: dynamic
 // scale from max|x| (amax words in ws, g written to g_out); mode 1: scale
 // read from g_in.
@@ -224,7 +235,7 @@ int run_quantize(DeviceState *d, const void *X, int64_t rows, int64_t K, int64_t
     p.zero = zero_word;
     const int64_t threads = rows_pad * groups * 4;
     int grid = static_cast<int>(std::min<int64_t>(std::max<int64_t>(cdiv(threads, 256), 1), int64_t(d->sm_count) * 16));
-    launch(nvfp4::quantize_kernel, dim3(grid), dim3(256), 0, stream, p);
+    launch_quantize(p, grid, stream);
     g_launches++;
     return launch_ok();
 }
@@ -255,7 +266,7 @@ int run_quantize_from_amax(DeviceState *d, const void *X, int64_t rows, int64_t 
     p.gate_up_F = 0;
     const int64_t threads = rows_pad * groups * 4;
     const int grid = static_cast<int>(std::min<int64_t>(std::max<int64_t>(cdiv(threads, 256), 1), int64_t(d->sm_count) * 16));
-    launch(nvfp4::quantize_kernel, dim3(grid), dim3(256), 0, stream, p);
+    launch_quantize(p, grid, stream);
     g_launches++;
     return launch_ok();
 }
@@ -781,7 +792,7 @@ int nvfp4_swiglu_quantize(const void *gate_up, int64_t M, int64_t F, int64_t ld,
     p.gate_up_F = 0;
     const int64_t threads = rows_pad * groups * 4;
     const int grid = static_cast<int>(std::min<int64_t>(std::max<int64_t>(cdiv(threads, 256), 1), int64_t(d->sm_count) * 16));
-    launch(nvfp4::quantize_kernel, dim3(grid), dim3(256), 0, s, p);
+    launch_quantize(p, grid, s);
     g_launches++;
     return launch_ok();
 }

@@ -185,6 +185,41 @@ __device__ __forceinline__ float global_scale_from_amax(uint32_t bits)
     return a == 0.0f ? 1.0f : __fdiv_rn(a, 2688.0f);
 }
 
+// E4M3 scale byte of a block whose largest magnitude is bamax:
+// s32 = fl32(fl32(bamax / 6) / g), by the shared-divisor division where it is
+// exact, then E4M3 round-to-nearest-even, saturating at 448.
+__device__ __forceinline__ uint32_t block_scale_byte(float bamax, float g, float rg, bool g_ok)
+{
+    float s32;
+    const float t_fast = div_shared(bamax, 6.0f, 0x1.555556p-3f /* RN(1/6) */);
+    if (g_ok && bamax >= 0x1p-17f && bamax <= 0x1p100f && div_shared_ok(g, t_fast))
+        s32 = div_shared(t_fast, g, rg);
+    else
+        s32 = __fdiv_rn(__fdiv_rn(bamax, 6.0f), g);
+    return f32_to_e4m3_satfinite(s32);
+}
+
+// Codes of a block outside the shared-divisor range: a zero decode scale
+// gives +-0 with the sign of each input, anything else the IEEE quotients.
+__device__ __forceinline__ void block_codes_slow(const uint32_t (&w)[8], float d, uint32_t (&packed)[2])
+{
+    packed[0] = packed[1] = 0u;
+    if (d == 0.0f) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const uint32_t lo = (w[i] >> 15) & 1u, hi = (w[i] >> 31) & 1u;
+            packed[i >> 2] |= ((lo << 3) | (hi << 7)) << ((i & 3) * 8);
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const float y0 = __fdiv_rn(bf16_lo(w[i]), d);
+            const float y1 = __fdiv_rn(bf16_hi(w[i]), d);
+            packed[i >> 2] |= f32x2_to_e2m1x2(y0, y1) << ((i & 3) * 8);
+        }
+    }
+}
+
 // Block scale and codes of one 16-element block held as two 16-byte words.
 // Returns the E4M3 scale byte and writes the 8 code bytes to packed[0..1].
 __device__ __forceinline__ uint32_t quantize_block(const uint4 &v0, const uint4 &v1, float g, float rg, bool g_ok,
@@ -192,25 +227,10 @@ __device__ __forceinline__ uint32_t quantize_block(const uint4 &v0, const uint4 
 {
     const uint32_t bmax = hmax16(vmax_mag(vmax_mag(0u, v0), v1));
     const float bamax = __uint_as_float(bmax << 16);
-    // s32 = fl32(fl32(bamax / 6) / g), by the shared-divisor division where it is exact
-    float s32;
-    const float t_fast = div_shared(bamax, 6.0f, 0x1.555556p-3f /* RN(1/6) */);
-    if (g_ok && bamax >= 0x1p-17f && bamax <= 0x1p100f && div_shared_ok(g, t_fast))
-        s32 = div_shared(t_fast, g, rg);
-    else
-        s32 = __fdiv_rn(__fdiv_rn(bamax, 6.0f), g);
-    const uint32_t sbyte = f32_to_e4m3_satfinite(s32);
+    const uint32_t sbyte = block_scale_byte(bamax, g, rg, g_ok);
     const float d = __fmul_rn(e4m3_to_f32(sbyte), g);
     const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-    packed[0] = packed[1] = 0u;
-    if (d == 0.0f) {
-        // zero scale: every code is +-0 with the sign of its input
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const uint32_t lo = (w[i] >> 15) & 1u, hi = (w[i] >> 31) & 1u;
-            packed[i >> 2] |= ((lo << 3) | (hi << 7)) << ((i & 3) * 8);
-        }
-    } else if (div_shared_ok(d, bamax)) {
+    if (d != 0.0f && div_shared_ok(d, bamax)) {
         const float nr = -__frcp_rn(d);
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
@@ -221,14 +241,23 @@ __device__ __forceinline__ uint32_t quantize_block(const uint4 &v0, const uint4 
             packed[h] = e2m1x8(y);
         }
     } else {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const float y0 = __fdiv_rn(bf16_lo(w[i]), d);
-            const float y1 = __fdiv_rn(bf16_hi(w[i]), d);
-            packed[i >> 2] |= f32x2_to_e2m1x2(y0, y1) << ((i & 3) * 8);
-        }
+        block_codes_slow(w, d, packed);
     }
     return sbyte;
+}
+
+// Eight E2M1 codes of the quotients x / d of the eight bf16 values in v (low
+// half of each word first), for a divisor in the shared-divisor range and
+// nr = -RN(1/d): the negated quotients are encoded and every code's sign bit
+// flipped back (div_shared_neg_x2).
+__device__ __forceinline__ uint32_t codes8_shared(const uint4 &v, float d, float nr)
+{
+    float y[8];
+    div_shared_neg_x2(v.x, d, nr, y[0], y[1]);
+    div_shared_neg_x2(v.y, d, nr, y[2], y[3]);
+    div_shared_neg_x2(v.z, d, nr, y[4], y[5]);
+    div_shared_neg_x2(v.w, d, nr, y[6], y[7]);
+    return e2m1x8(y) ^ 0x88888888u;
 }
 
 // Work item = one 512-element chunk of one row (32 blocks = 8 scale words),
@@ -303,6 +332,101 @@ __global__ void __launch_bounds__(256) quantize_kernel(const QuantParams p)
             const uint32_t srow = stored_row(p, row);
             const uint64_t tile = static_cast<uint64_t>(srow >> 7) * p.groups + cg;
             const uint32_t rr = srow & 127u;
+            *reinterpret_cast<uint32_t *>(p.sf + tile * 512 + (rr & 31u) * 16 + (rr >> 5) * 4) = word;
+        }
+        row = nrow;
+        chunk = nchunk;
+        v0 = n0;
+        v1 = n1;
+    }
+}
+
+// quantize_kernel for one module segment with rows stored in order (every
+// activation): the same work items and the same results.  The decode scale
+// d = fl32(s g), nr = -RN(1/d) and the largest block amax for which the
+// shared-divisor quotients are exact (d 2^100) depend only on the block's
+// scale byte s, so each CTA tabulates them once for the 127 finite bytes and
+// a block looks its entry up instead of decoding s and taking a correctly
+// rounded reciprocal; the quotients are taken on the unnegated inputs
+// (codes8_shared).
+__global__ void __launch_bounds__(256) quantize_act_kernel(const QuantParams p)
+{
+    grid_dep_wait();
+    grid_dep_launch_dependents();
+    __shared__ float4 s_tab[128];  // {d, nr, d 2^100 or -1 outside the shared-divisor range, 0}
+    const float g = (p.mode == 0) ? global_scale_from_amax(p.amax_bits[0]) : p.g_in[0];
+    if (threadIdx.x < 128) {
+        // byte 0x7F is E4M3's NaN; the saturating conversion never produces it
+        const float d = __fmul_rn(e4m3_to_f32(threadIdx.x), g);
+        const bool fast = threadIdx.x < 127 && d >= 0x1p-80f && d <= 0x1p100f;
+        s_tab[threadIdx.x] =
+            make_float4(d, fast ? -__frcp_rn(d) : 0.0f, fast ? __fmul_rn(d, 0x1p100f) : -1.0f, 0.0f);
+    }
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+        if (p.zero != nullptr)
+            *p.zero = 0;
+        if (p.mode == 0 && p.g_out != nullptr)
+            p.g_out[0] = g;
+    }
+    const float rg = __frcp_rn(g);
+    const bool g_ok = g >= 0x1p-80f && g <= 0x1p100f;
+    __syncthreads();
+
+    const int lane = threadIdx.x & 31;
+    const uint32_t cpr = (static_cast<uint32_t>(p.groups) + 7u) >> 3;  // chunks per row
+    const uint32_t items = static_cast<uint32_t>(p.rows_pad) * cpr;
+    const uint32_t warp0 = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const uint32_t nwarps = (gridDim.x * blockDim.x) >> 5;
+    const uint32_t drow = nwarps / cpr, dchunk = nwarps - drow * cpr;
+    const int nblk = p.K >> 4;
+    const uint32_t rows = static_cast<uint32_t>(p.rows);
+
+    uint32_t row = warp0 / cpr, chunk = warp0 - row * cpr;
+    auto load = [&](uint32_t r, uint32_t c, uint4 &a, uint4 &b) {
+        const int blk = static_cast<int>(c * 32u) + lane;
+        if (r < rows && blk < nblk) {
+            const uint4 *src = reinterpret_cast<const uint4 *>(p.X + static_cast<int64_t>(r) * p.ld + blk * 16);
+            a = __ldg(src);
+            b = __ldg(src + 1);
+        }
+    };
+    uint4 v0 = make_uint4(0, 0, 0, 0), v1 = v0;
+    if (warp0 < items)
+        load(row, chunk, v0, v1);
+    for (uint32_t item = warp0; item < items; item += nwarps) {
+        uint32_t nrow = row + drow, nchunk = chunk + dchunk;
+        if (nchunk >= cpr) {
+            nchunk -= cpr;
+            ++nrow;
+        }
+        uint4 n0 = make_uint4(0, 0, 0, 0), n1 = n0;
+        if (item + nwarps < items)
+            load(nrow, nchunk, n0, n1);
+
+        const int blk = static_cast<int>(chunk * 32u) + lane;
+        uint32_t sbyte = 0;
+        if (row < rows && blk < nblk) {
+            const float bamax = __uint_as_float(hmax16(vmax_mag(vmax_mag(0u, v0), v1)) << 16);
+            sbyte = block_scale_byte(bamax, g, rg, g_ok);
+            const float4 e = s_tab[sbyte];
+            uint32_t packed[2];
+            if (bamax <= e.z) {
+                packed[0] = codes8_shared(v0, e.x, e.y);
+                packed[1] = codes8_shared(v1, e.x, e.y);
+            } else {
+                const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+                block_codes_slow(w, e.x, packed);
+            }
+            *reinterpret_cast<uint2 *>(p.codes + static_cast<int64_t>(row) * (p.K >> 1) + blk * 8) =
+                make_uint2(packed[0], packed[1]);
+        }
+        // four neighbouring blocks -> one 32-bit scale word, in lanes 0, 4, 8, ...
+        const uint32_t pair = sbyte | (__shfl_down_sync(0xFFFFFFFFu, sbyte, 1) << 8);
+        const uint32_t word = pair | (__shfl_down_sync(0xFFFFFFFFu, pair, 2) << 16);
+        const uint32_t cg = chunk * 8u + (lane >> 2);
+        if ((lane & 3) == 0 && cg < static_cast<uint32_t>(p.groups)) {
+            const uint64_t tile = static_cast<uint64_t>(row >> 7) * p.groups + cg;
+            const uint32_t rr = row & 127u;
             *reinterpret_cast<uint32_t *>(p.sf + tile * 512 + (rr & 31u) * 16 + (rr >> 5) * 4) = word;
         }
         row = nrow;

@@ -1,6 +1,7 @@
-// Compares the quantizer's shared-divisor division (div_shared and its packed
-// two-lane form div_shared_x2, from fp_div.cuh) with CUDA's IEEE division
-// __fdiv_rn, bit for bit (div_shared_x2 on the pair (x, -x)):
+// Compares the quantizer's shared-divisor division (div_shared, its packed
+// two-lane form div_shared_x2 and the negated form div_shared_neg_x2, from
+// fp_div.cuh) with CUDA's IEEE division __fdiv_rn, bit for bit (the packed
+// forms on the pair (x, -x); div_shared_neg_x2 against -__fdiv_rn):
 //  (1) every bf16 significand x (128) against every fp32 significand d (2^23),
 //      with exponents chosen so x/d spans [2^-5, 2^5), both signs;
 //  (2) every finite bf16 value against pseudo-random divisors over the whole
@@ -15,6 +16,7 @@
 using nvfp4::div_shared;
 using nvfp4::div_shared_ok;
 using nvfp4::div_shared_x2;
+using nvfp4::div_shared_neg_x2;
 
 // bf16 bits of x (x is a bf16 value) in the low half, of -x in the high half
 __device__ uint32_t pair_of(float x)
@@ -71,6 +73,14 @@ __global__ void sweep_significands(unsigned long long *checked, unsigned long lo
                             record(xs, d, y2lo, ref);
                         }
                         c += 2;
+                        float n2lo, n2hi;
+                        div_shared_neg_x2(pair_of(xs), d, -r, n2lo, n2hi);
+                        if (__float_as_uint(n2lo) != (__float_as_uint(ref) ^ 0x80000000u) ||
+                            __float_as_uint(n2hi) != (__float_as_uint(ref_neg) ^ 0x80000000u)) {
+                            ++b;
+                            record(xs, d, -n2lo, ref);
+                        }
+                        c += 2;
                     }
                 }
             }
@@ -102,13 +112,14 @@ __global__ void sweep_range(unsigned long long *checked, unsigned long long *bad
             continue;
         ++a;
         const float r = __frcp_rn(d);
-        float y2[2];
+        float y2[2], n2[2];
         div_shared_x2(pair_of(x), d, -r, y2[0], y2[1]);
-        const float ys[3] = {div_shared(x, d, r), y2[0], y2[1]};
-        const float refs[3] = {__fdiv_rn(x, d), __fdiv_rn(x, d), __fdiv_rn(-x, d)};
+        div_shared_neg_x2(pair_of(x), d, -r, n2[0], n2[1]);
+        const float ys[5] = {div_shared(x, d, r), y2[0], y2[1], -n2[0], -n2[1]};
+        const float refs[5] = {__fdiv_rn(x, d), __fdiv_rn(x, d), __fdiv_rn(-x, d), __fdiv_rn(x, d), __fdiv_rn(-x, d)};
         // quotients >= 2^-20 must be the IEEE ones; smaller ones must stay below
         // 0.25 (all encode to +-0) with the sign of x
-        for (int k = 0; k < 3; ++k) {
+        for (int k = 0; k < 5; ++k) {
             const float y = ys[k], ref = refs[k];
             if (fabsf(ref) >= 0x1p-20f || fabsf(y) >= 0x1p-20f) {
                 if (__float_as_uint(y) != __float_as_uint(ref)) {
