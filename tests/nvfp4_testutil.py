@@ -11,6 +11,38 @@ from nvfp4_w4a4_quantized_act_b200 import workloads as wl
 
 DEV = "cuda"
 
+GUARD_BYTES = 4096
+SENTINEL = 0xA5
+
+
+class Guarded:
+    """A device buffer with GUARD_BYTES of sentinel bytes on each side: the
+    bounds check that stands in for a memory sanitizer.  `t` is the buffer a
+    call may write (16-byte aligned, contiguous); check() asserts that no
+    byte around it changed."""
+
+    def __init__(self, shape, dtype, fill=None, device=DEV):
+        shape = tuple(shape) if isinstance(shape, (tuple, list)) else (int(shape),)
+        n = 1
+        for d in shape:
+            n *= int(d)
+        nbytes = n * torch.empty((), dtype=dtype).element_size()
+        self.raw = torch.full((2 * GUARD_BYTES + nbytes,), SENTINEL, dtype=torch.uint8, device=device)
+        self.t = self.raw[GUARD_BYTES: GUARD_BYTES + nbytes].view(dtype).view(shape)
+        if fill is not None:
+            self.t.fill_(fill)
+
+    def check(self, what: str = ""):
+        if self.raw.is_cuda:
+            torch.cuda.synchronize()
+        head = self.raw[:GUARD_BYTES]
+        tail = self.raw[self.raw.numel() - GUARD_BYTES:]
+        bad_head = int((head != SENTINEL).sum())
+        bad_tail = int((tail != SENTINEL).sum())
+        assert bad_head == 0 and bad_tail == 0, (
+            f"{what}: {bad_head} bytes before and {bad_tail} bytes after the buffer were written")
+        return self.t
+
 
 def dev_u8(a: np.ndarray) -> torch.Tensor:
     return torch.from_numpy(np.ascontiguousarray(a).reshape(-1).view(np.uint8)).to(DEV)
@@ -107,15 +139,22 @@ def oracle_sampled(xb, wb, segments, ms, ns):
 def full_size_check(X, W, segments, seed):
     """nvfp4_linear_fused at full size (bf16 and fp32 outputs) against the
     oracle on sampled outputs; the quantized operands of the sampled rows
-    are checked bit for bit.  Returns the largest error / tolerance ratio."""
+    are checked bit for bit and the bytes around the outputs and the
+    workspace must be untouched.  Returns the largest error / tolerance
+    ratio."""
     M, K = X.shape
     N = W.shape[0]
     xb, wb = wl.bf16_bits(X), wl.bf16_bits(W)
     qw = ops.quantize_weights(W.to(DEV), segments)
     Xd = X.to(DEV)
-    ws = torch.empty(ops.workspace_bytes(M, N, K, len(segments)), dtype=torch.uint8, device=DEV)
-    out = ops.linear_fused(Xd, qw, ws=ws)
-    out32 = ops.linear_fused(Xd, qw, ws=ws, out_fp32=True)
+    gws = Guarded(ops.workspace_bytes(M, N, K, len(segments)), torch.uint8)
+    ws = gws.t
+    g16 = Guarded((M, N), torch.bfloat16)
+    g32 = Guarded((M, N), torch.float32)
+    ops.linear_fused(Xd, qw, out=g16.t, ws=ws)
+    ops.linear_fused(Xd, qw, out=g32.t, ws=ws, out_fp32=True)
+    out, out32 = g16.check("bf16 output"), g32.check("fp32 output")
+    gws.check("workspace")
     assert ops.get_status() == 0
     rng = np.random.default_rng(seed)
     ms, ns = sample_outputs(M, N, segments, rng)

@@ -24,6 +24,7 @@ BUDGET = {
     "gemm_nvf4_kernel<false>": (168, 0, 0),
     "splitk_finalize_kernel": (255, 0, 0),
     "quantize_kernel": (64, 0, 0),
+    "quantize_act_kernel": (64, 0, 0),
     "amax_kernel": (64, 0, 0),
     "swiglu_kernel": (64, 0, 0),
     "kv_quantize_kernel": (64, 0, 0),

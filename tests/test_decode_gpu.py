@@ -3,7 +3,9 @@ tile's K steps among several CTAs (split-K) and sums the fp32 partials in a
 fixed order: every output against the oracle on all rows (all columns, or
 sampled columns plus every module boundary for wide fused weights), bf16 =
 RNE(fp32), run-to-run bit equality, the unsplit GEMM on the same quantized
-activation within the same tolerance, and the launch that does the sum."""
+activation within the same tolerance, and the launch that does the sum.  No
+byte around the outputs and workspaces (where the split-K partials live) may
+change."""
 import numpy as np
 import pytest
 import torch
@@ -11,7 +13,7 @@ import torch
 import oracle
 from nvfp4_w4a4_quantized_act_b200 import ops
 from nvfp4_w4a4_quantized_act_b200 import workloads as wl
-from nvfp4_testutil import DEV, bf16_of_f32, check_gemm, host
+from nvfp4_testutil import DEV, Guarded, bf16_of_f32, check_gemm, host
 
 pytestmark = pytest.mark.gpu
 
@@ -51,9 +53,15 @@ def test_decode_linear_matches_oracle(M, N, K, widths):
     xb, wb = wl.bf16_bits(X), wl.bf16_bits(W)
     qw = ops.quantize_weights(W.to(DEV), segs)
     Xd = X.to(DEV)
-    ws = torch.empty(ops.workspace_bytes(M, N, K, len(segs)), dtype=torch.uint8, device=DEV)
-    out32 = host(ops.linear_fused(Xd, qw, out_fp32=True, ws=ws))
-    out16 = host(ops.linear_fused(Xd, qw, ws=ws).view(torch.int16)).view(np.uint16)
+    gws = Guarded(ops.workspace_bytes(M, N, K, len(segs)), torch.uint8)
+    ws = gws.t
+    g32 = Guarded((M, N), torch.float32, fill=float("nan"))
+    g16 = Guarded((M, N), torch.bfloat16, fill=float("nan"))
+    ops.linear_fused(Xd, qw, out=g32.t, out_fp32=True, ws=ws)
+    ops.linear_fused(Xd, qw, out=g16.t, ws=ws)
+    out32 = host(g32.check("fp32 output"))
+    out16 = host(g16.check("bf16 output").view(torch.int16)).view(np.uint16)
+    gws.check("workspace (activation codes, scales, split-K partials)")
     again = host(ops.linear_fused(Xd, qw, out_fp32=True, ws=ws))
     assert ops.get_status() == 0
 
@@ -73,8 +81,11 @@ def test_decode_linear_matches_oracle(M, N, K, widths):
     assert ops.get_status() == 0
     check_gemm(plain[:, cols], C, B, "unsplit")
     # the workspace form splits like the linear: the same bits on the same operands
-    gws = torch.empty(max(ops.gemm_workspace_bytes(M, N, K), 16), dtype=torch.uint8, device=DEV)
-    pre = host(ops.gemm_prequant(c_ws, sf_ws, g_ws, M, K, qw, out_fp32=True, ws=gws))
+    gpw = Guarded(max(ops.gemm_workspace_bytes(M, N, K), 16), torch.uint8)
+    gpo = Guarded((M, N), torch.float32, fill=float("nan"))
+    ops.gemm_prequant(c_ws, sf_ws, g_ws, M, K, qw, out=gpo.t, out_fp32=True, ws=gpw.t)
+    pre = host(gpo.check("pre-quantized GEMM output"))
+    gpw.check("split-K workspace")
     assert ops.get_status() == 0
     assert np.array_equal(pre, out32)
 

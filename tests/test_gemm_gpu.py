@@ -1,7 +1,8 @@
 """Block-scaled FP4 GEMM on the tensor cores against the oracle's fp64 GEMM
 over the same (oracle-quantized) operands: every output within
 1e-5 * sum|a*b| + 1e-6; bf16 outputs equal the RNE rounding of the fp32
-path; exact-integer problems bit-exact.  Shapes with M > 128 run on the
+path; exact-integer problems bit-exact; no byte around an output buffer
+is written (ragged tiles clipped at the edges).  Shapes with M > 128 run on the
 CTA-pair kernel by default; each check also runs the one-CTA kernel
 (NVFP4_SINGLE_CTA) on the same operands."""
 import numpy as np
@@ -11,7 +12,7 @@ import torch
 import oracle
 from nvfp4_w4a4_quantized_act_b200 import ops
 from nvfp4_w4a4_quantized_act_b200 import workloads as wl
-from nvfp4_testutil import (DEV, bf16_of_f32, check_gemm, dev_u8, host, oracle_act_on_device,
+from nvfp4_testutil import (DEV, Guarded, bf16_of_f32, check_gemm, dev_u8, host, oracle_act_on_device,
                             oracle_weight_on_device)
 
 pytestmark = pytest.mark.gpu
@@ -24,9 +25,12 @@ def _run(xb, wb, segments, flags=0):
     M, K = xb.shape
     (ac, asf, ga), (oc, os_, og) = oracle_act_on_device(xb)
     qw, (wc, ws, wg) = oracle_weight_on_device(wb, segments)
-    out32 = ops.gemm_prequant(ac, asf, ga, M, K, qw, out_fp32=True, debug_flags=flags)
-    out16 = ops.gemm_prequant(ac, asf, ga, M, K, qw, debug_flags=flags)
-    torch.cuda.synchronize()
+    g32 = Guarded((M, wb.shape[0]), torch.float32, fill=float("nan"))
+    g16 = Guarded((M, wb.shape[0]), torch.bfloat16, fill=float("nan"))
+    ops.gemm_prequant(ac, asf, ga, M, K, qw, out=g32.t, out_fp32=True, debug_flags=flags)
+    ops.gemm_prequant(ac, asf, ga, M, K, qw, out=g16.t, debug_flags=flags)
+    out32 = g32.check("fp32 output")
+    out16 = g16.check("bf16 output")
     grow = oracle.rows_scale(segments, wg, wb.shape[0])
     C, B = oracle.linear_full(oc, os_, og, wc, ws, grow)
     return host(out32), host(out16.view(torch.int16)).view(np.uint16), C, B

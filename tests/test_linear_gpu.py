@@ -8,7 +8,7 @@ import torch
 import oracle
 from nvfp4_w4a4_quantized_act_b200 import ops
 from nvfp4_w4a4_quantized_act_b200 import workloads as wl
-from nvfp4_testutil import DEV, bf16_of_f32, check_gemm, full_size_check, host
+from nvfp4_testutil import DEV, Guarded, bf16_of_f32, check_gemm, full_size_check, host
 
 pytestmark = pytest.mark.gpu
 
@@ -46,8 +46,9 @@ def test_fused_matches_oracle_and_concat_of_modules():
     M, K = 300, 512
     X = wl.activation_normal(M, K, 8)
     qw = ops.quantize_weights(W.to(DEV), segs)
-    fused = ops.linear_fused(X.to(DEV), qw, out_fp32=True)
-    torch.cuda.synchronize()
+    gout = Guarded((M, W.shape[0]), torch.float32, fill=float("nan"))
+    fused = ops.linear_fused(X.to(DEV), qw, out=gout.t, out_fp32=True)
+    gout.check("fused output")
     ca, sa, ga = oracle.quantize_tensor(wl.bf16_bits(X))
     cw, sw, gseg = oracle.quantize_segments(wl.bf16_bits(W), segs)
     C, B = oracle.linear_full(ca, sa, ga, cw, sw, oracle.rows_scale(segs, gseg, W.shape[0]))

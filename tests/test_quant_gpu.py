@@ -1,6 +1,6 @@
 """Activation / weight quantization on the GPU against the oracle: packed
 codes, swizzled scale bytes (padding included) and global scales must match
-bit for bit."""
+bit for bit, and no byte around the codes and scale buffers may change."""
 import numpy as np
 import pytest
 import torch
@@ -8,14 +8,18 @@ import torch
 import oracle
 from nvfp4_w4a4_quantized_act_b200 import ops
 from nvfp4_w4a4_quantized_act_b200 import workloads as wl
-from nvfp4_testutil import DEV, dev_u8, host
+from nvfp4_testutil import DEV, Guarded, dev_u8, host
 
 pytestmark = pytest.mark.gpu
 
 
 def _gpu_quant(X: torch.Tensor):
-    codes, sf, g = ops.quantize_act(X.to(DEV))
-    torch.cuda.synchronize()
+    M, K = X.shape
+    gc = Guarded(M * K // 2, torch.uint8, fill=0x5A)
+    gs = Guarded(ops.sf_bytes(M, K), torch.uint8, fill=0x5A)
+    codes, sf, g = ops.quantize_act(X.to(DEV), codes=gc.t, sf=gs.t)
+    gc.check("codes")
+    gs.check("scale factors")
     return host(codes), host(sf), float(host(g)[0])
 
 

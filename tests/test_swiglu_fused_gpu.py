@@ -2,7 +2,8 @@
 (nvfp4_quantize_weights_gated + nvfp4_linear_swiglu) against the oracle:
 the interleaved weight layout and the quantized operands bit for bit, h
 within the GEMM tolerance carried through silu(g)*u plus bf16 rounding, and
-the requantization of the GPU's own h bit for bit."""
+the requantization of the GPU's own h bit for bit; no byte around h, its
+codes, scales or the workspace may change."""
 import numpy as np
 import pytest
 import torch
@@ -10,7 +11,7 @@ import torch
 import oracle
 from nvfp4_w4a4_quantized_act_b200 import ops
 from nvfp4_w4a4_quantized_act_b200 import workloads as wl
-from nvfp4_testutil import DEV, host
+from nvfp4_testutil import DEV, Guarded, host
 
 pytestmark = pytest.mark.gpu
 
@@ -46,7 +47,14 @@ def _h_tolerance(Cg, Bg, Cu, Bu, h_ref):
 
 def _check(M, K, F, X, W, rows, cols, single_cta=False):
     qw = ops.quantize_weights_gated(W.to(DEV))
-    h, hc, hsf, gh = ops.linear_swiglu(X.to(DEV), qw, single_cta=single_cta)
+    gh_ = Guarded((M, F), torch.bfloat16, fill=float("nan"))
+    gc_ = Guarded(M * F // 2, torch.uint8, fill=0x5A)
+    gs_ = Guarded(ops.sf_bytes(M, F), torch.uint8, fill=0x5A)
+    gw_ = Guarded(ops.workspace_bytes(M, 2 * F, K, 2), torch.uint8)
+    h, hc, hsf, gh = ops.linear_swiglu(X.to(DEV), qw, h=gh_.t, h_codes=gc_.t, h_sf=gs_.t, ws=gw_.t,
+                                       single_cta=single_cta)
+    for g, what in ((gh_, "h"), (gc_, "h codes"), (gs_, "h scale factors"), (gw_, "workspace")):
+        g.check(what)
     assert ops.get_status() == 0
     xb, wb = wl.bf16_bits(X), wl.bf16_bits(W)
     g_a = oracle.global_scale(oracle.amax(xb))
