@@ -45,7 +45,7 @@ def test_tiny_linear_operands_bit_exact():
     _assert_same(W)
 
 
-@pytest.mark.parametrize("M,K", [(1, 16), (7, 48), (130, 64), (257, 272), (64, 320), (300, 1024), (33, 5120)])
+@pytest.mark.parametrize("M,K", [(1, 16), (7, 48), (3, 80), (130, 64), (257, 272), (64, 320), (300, 1024), (33, 5120)])
 def test_ragged_shapes_bit_exact(M, K):
     _assert_same(wl.activation_normal(M, K, seed=M * 31 + K, n_outliers=min(4, K // 16), scale=50.0))
 
