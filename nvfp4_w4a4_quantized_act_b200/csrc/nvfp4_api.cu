@@ -196,8 +196,10 @@ int run_amax(DeviceState *d, const void *X, int64_t rows, int64_t K, int64_t ld,
 // row order.
 void launch_quantize(const nvfp4::QuantParams &p, int grid, cudaStream_t stream)
 {
-    if (p.seg.nseg == 1 && p.gate_up_F == 0)
-        launch(nvfp4::quantize_act_kernel, dim3(grid), dim3(256), 0, stream, p);
+    if (p.seg.nseg == 1 && p.gate_up_F == 0 && p.mode == 2)
+        launch(nvfp4::quantize_act_kernel<true>, dim3(grid), dim3(256), 0, stream, p);
+    else if (p.seg.nseg == 1 && p.gate_up_F == 0)
+        launch(nvfp4::quantize_act_kernel<false>, dim3(grid), dim3(256), 0, stream, p);
     else
         launch(nvfp4::quantize_kernel, dim3(grid), dim3(256), 0, stream, p);
 }
@@ -215,7 +217,12 @@ int run_quantize(DeviceState *d, const void *X, int64_t rows, int64_t K, int64_t
     const int64_t groups = cdiv(K, 64);
     if (rows_pad * groups * 4 >= (int64_t(1) << 31) || K > (int64_t(1) << 30))
         return NVFP4_ERR_UNSUPPORTED_SHAPE;
-    if (dynamic && run_amax(d, X, rows, K, ld, seg, amax_ws, stream) != NVFP4_OK)
+    // a decode-sized activation (at most 32 KB): every quantize CTA takes
+    // max|x| itself, one launch instead of the one-CTA amax pass and the
+    // quantize (at 16 tokens, where every CTA would read 160-192 KB, that was
+    // much slower)
+    const bool cta_amax = dynamic && seg.nseg == 1 && gate_up_F == 0 && rows > 0 && rows * K * 2 <= kOneBlockAmaxBytes;
+    if (dynamic && !cta_amax && run_amax(d, X, rows, K, ld, seg, amax_ws, stream) != NVFP4_OK)
         return NVFP4_ERR_CUDA;
     nvfp4::QuantParams p;
     p.X = static_cast<const uint16_t *>(X);
@@ -228,7 +235,8 @@ int run_quantize(DeviceState *d, const void *X, int64_t rows, int64_t K, int64_t
     p.amax_bits = amax_ws;
     p.g_in = g_in;
     p.g_out = g_out;
-    p.mode = dynamic ? 0 : 1;
+    p.mode = cta_amax ? 2 : (dynamic ? 0 : 1);
+    p.status = d->status;
     p.codes = codes;
     p.sf = sf;
     p.gate_up_F = static_cast<int32_t>(gate_up_F);

@@ -157,8 +157,9 @@ struct QuantParams {
     SegRows seg;
     const uint32_t *amax_bits;  // mode 0: per-segment amax bits
     const float *g_in;          // mode 1: per-segment global scale
-    float *g_out;               // mode 0: per-segment global scale written here (may be null)
-    int32_t mode;
+    float *g_out;               // modes 0, 2: per-segment global scale written here (may be null)
+    int32_t mode;               // 0: g from amax_bits, 1: g given, 2: g from max|x| taken by every CTA
+    uint32_t *status = nullptr; // mode 2: latched error bits (non-finite input)
     uint8_t *codes;          // [rows, K/2]
     uint8_t *sf;             // swizzled scale tiles
     int32_t gate_up_F;       // > 0: rows are [gate F | up F]; stored interleaved in 128-row blocks
@@ -349,12 +350,39 @@ __global__ void __launch_bounds__(256) quantize_kernel(const QuantParams p)
 // a block looks its entry up instead of decoding s and taking a correctly
 // rounded reciprocal; the quotients are taken on the unnegated inputs
 // (codes8_shared).
+template <bool CTA_AMAX = false>
 __global__ void __launch_bounds__(256) quantize_act_kernel(const QuantParams p)
 {
     grid_dep_wait();
     grid_dep_launch_dependents();
     __shared__ float4 s_tab[128];  // {d, nr, d 2^100 or -1 outside the shared-divisor range, 0}
-    const float g = (p.mode == 0) ? global_scale_from_amax(p.amax_bits[0]) : p.g_in[0];
+    __shared__ uint32_t s_amax;
+    float g;
+    if (CTA_AMAX) {
+        // mode 2, a decode-sized input: every CTA reads all of it (from L2) for max|x|,
+        // so the global scale needs neither an amax launch nor a grid barrier
+        if (threadIdx.x == 0)
+            s_amax = 0;
+        __syncthreads();
+        const int64_t cpr16 = p.K >> 3;  // 16-byte chunks per row
+        uint32_t m = 0;
+        for (int64_t i = threadIdx.x; i < static_cast<int64_t>(p.rows) * cpr16; i += blockDim.x) {
+            const int64_t r = i / cpr16, c = i - r * cpr16;
+            m = vmax_mag(m, __ldg(reinterpret_cast<const uint4 *>(p.X + r * p.ld) + c));
+        }
+        uint32_t v = hmax16(m);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+            v = max(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
+        if ((threadIdx.x & 31) == 0 && v != 0)
+            atomicMax(&s_amax, v);
+        __syncthreads();
+        if (blockIdx.x == 0 && threadIdx.x == 0 && s_amax >= 0x7F80u)  // Inf or NaN magnitude
+            atomicOr(p.status, kStatusNonFinite);
+        g = global_scale_from_amax(s_amax);
+    } else {
+        g = (p.mode == 0) ? global_scale_from_amax(p.amax_bits[0]) : p.g_in[0];
+    }
     if (threadIdx.x < 128) {
         // byte 0x7F is E4M3's NaN; the saturating conversion never produces it
         const float d = __fmul_rn(e4m3_to_f32(threadIdx.x), g);
@@ -365,7 +393,7 @@ __global__ void __launch_bounds__(256) quantize_act_kernel(const QuantParams p)
     if (blockIdx.x == 0 && threadIdx.x == 0) {
         if (p.zero != nullptr)
             *p.zero = 0;
-        if (p.mode == 0 && p.g_out != nullptr)
+        if (p.mode != 1 && p.g_out != nullptr)
             p.g_out[0] = g;
     }
     const float rg = __frcp_rn(g);

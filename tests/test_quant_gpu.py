@@ -117,13 +117,14 @@ def test_weights_per_segment_bit_exact():
     assert np.array_equal(host(qw.sf), oracle.swizzle(s_ref, 256))
 
 
-def test_nonfinite_input_is_reported():
-    x = np.ones((128, 64), dtype=np.float32)
+@pytest.mark.parametrize("M,K", [(128, 64), (1024, 512)])  # every CTA takes max|x| / a separate amax pass
+def test_nonfinite_input_is_reported(M, K):
+    x = np.ones((M, K), dtype=np.float32)
     x[5, 7] = np.inf
     ops.quantize_act(wl.to_bf16(x).to(DEV))
     assert ops.get_status() == 6
     assert ops.get_status() == 0  # cleared
-    ops.quantize_act(torch.ones((128, 64), dtype=torch.bfloat16, device=DEV))
+    ops.quantize_act(torch.ones((M, K), dtype=torch.bfloat16, device=DEV))
     assert ops.get_status() == 0
 
 
