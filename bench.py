@@ -48,25 +48,44 @@ FP4_PER_BF16 = 4.0  # dense FP4 : dense BF16 tensor throughput on B200 (9 : 2.25
 FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # DRAM bytes (read + write) per GEMM launch, mean over the four GEMM launches of
 # one layer, from one ncu capture (the DRAM-bytes capture of these sources).
-# Reported only while the GEMM kernel sources and the host code that sets up
-# their launches (tile order, grid, tensor-map boxes, split-K) still hash to
-# the captured value.
-GEMM_TRAFFIC = {"source_sha256_12": "899458b90972", "bytes_per_launch": 275.78e6}
-GEMM_SOURCES = [os.path.join(ROOT, "nvfp4_w4a4_quantized_act_b200", "csrc", f)
-                for f in ("gemm_kernel.cuh", "gemm_pair_kernel.cuh", "ptx_sm100.cuh", "nvfp4_api.cu")]
+# Reported only while the GEMM kernel sources and the host functions that set
+# up their launches (tile order, grid, tensor-map boxes) still hash to the
+# captured value.
+GEMM_TRAFFIC = {"source_sha256_12": "8a6aa8e168f6", "bytes_per_launch": 275.78e6}
+_CSRC = os.path.join(ROOT, "nvfp4_w4a4_quantized_act_b200", "csrc")
+# (file, None for the whole file, or the functions of it that configure GEMM launches)
+GEMM_SOURCES = [(os.path.join(_CSRC, "gemm_kernel.cuh"), None),
+                (os.path.join(_CSRC, "gemm_pair_kernel.cuh"), None),
+                (os.path.join(_CSRC, "ptx_sm100.cuh"), None),
+                (os.path.join(_CSRC, "nvfp4_api.cu"), ("make_codes_map", "make_sf_map", "make_out_map", "run_gemm"))]
+
+
+def _function_text(text, name):
+    """Source of the top-level function `name` (its signature line through the
+    first closing brace in column 0)."""
+    import re
+    m = re.search(r"^[A-Za-z_][^\n;]*\b" + re.escape(name) + r"\(", text, flags=re.M)
+    if m is None:
+        raise ValueError(f"function {name} not found")
+    end = text.index("\n}\n", m.start())
+    return text[m.start(): end + 3]
 
 
 def gemm_source_hash():
-    """Hash of the GEMM kernel sources with comments and whitespace removed,
-    so that an edit to a comment keeps the captured traffic valid."""
+    """Hash of the GEMM sources with comments and whitespace removed, so that
+    an edit to a comment (or to code outside the listed functions) keeps the
+    captured traffic valid."""
     import hashlib
     import re
     h = hashlib.sha256()
-    for path in GEMM_SOURCES:
+    for entry in GEMM_SOURCES:
+        path, funcs = entry if isinstance(entry, tuple) else (entry, None)
         with open(path) as f:
             text = f.read()
         text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
         text = re.sub(r"//[^\n]*", " ", text)
+        if funcs is not None:
+            text = "\n".join(_function_text(text, fn) for fn in funcs)
         h.update(" ".join(text.split()).encode())
     return h.hexdigest()[:12]
 

@@ -68,12 +68,23 @@ def test_gemm_source_hash_ignores_comments_only(tmp_path, monkeypatch):
     assert bench.gemm_traffic() is None
 
 
-def test_gemm_source_hash_covers_the_launch_code():
-    """The hash also covers the host code that chooses the GEMM's tile
-    order, grid, tensor-map boxes and split-K (nvfp4_api.cu): a change
-    there invalidates the captured traffic too."""
+def test_gemm_source_hash_covers_the_launch_code(tmp_path, monkeypatch):
+    """The hash also covers the host functions that choose the GEMM's tile
+    order, grid and tensor-map boxes (run_gemm and the tensor-map builders in
+    nvfp4_api.cu): a change there invalidates the captured traffic, a change
+    elsewhere in that file does not."""
     import bench
-    names = [os.path.basename(p) for p in bench.GEMM_SOURCES]
-    assert "nvfp4_api.cu" in names
-    assert {"gemm_kernel.cuh", "gemm_pair_kernel.cuh", "ptx_sm100.cuh"} <= set(names)
-    assert all(os.path.exists(p) for p in bench.GEMM_SOURCES)
+    entries = {os.path.basename(p): f for p, f in bench.GEMM_SOURCES}
+    assert {"gemm_kernel.cuh", "gemm_pair_kernel.cuh", "ptx_sm100.cuh", "nvfp4_api.cu"} <= set(entries)
+    assert "run_gemm" in entries["nvfp4_api.cu"]
+    assert all(os.path.exists(p) for p, _ in bench.GEMM_SOURCES)
+    src = tmp_path / "api.cu"
+    body = ("int other(int a)\n{\n    return a + 1;\n}\n\n"
+            "int run_gemm(int m, int n)\n{\n    const int grid = m * n;\n    return grid;\n}\n")
+    src.write_text(body)
+    monkeypatch.setattr(bench, "GEMM_SOURCES", [(str(src), ("run_gemm",))])
+    h0 = bench.gemm_source_hash()
+    src.write_text(body.replace("a + 1", "a + 2"))
+    assert bench.gemm_source_hash() == h0
+    src.write_text(body.replace("m * n", "m * n + 1"))
+    assert bench.gemm_source_hash() != h0
