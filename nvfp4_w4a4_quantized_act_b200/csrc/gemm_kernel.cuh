@@ -88,6 +88,9 @@ struct Params {
     int32_t splits;
     int32_t kt_per_split;
     float *partial;
+    // the partials of a CTA's last work item go out through shared memory,
+    // a row per store instruction (store_partial_staged); set for M >= 64
+    int32_t staged_partials;
     // the weight producer may load before the previous kernel on the stream
     // has finished (that kernel does not write W)
     int32_t w_early;
@@ -254,6 +257,50 @@ __device__ __forceinline__ void store_partial_64(const Params &p, int split, con
         for (int j = 0; j < 64 && col0 + j < p.N; ++j)
             o[j] = __fmul_rn(__uint_as_float(v[j]), alpha[j]);
     }
+}
+
+// Staging rows of store_partial_staged: 64 values + 4 of padding, so that
+// the 16-byte writes of a warp spread over the shared-memory banks.
+constexpr int STG_LD = 68;
+constexpr uint32_t STG_WARP_BYTES = 32 * STG_LD * 4;
+static_assert((EPI_THREADS / 32) * STG_WARP_BYTES <= STAGES * STAGE_BYTES, "staging rows fit in the pipeline ring");
+
+// Split-K partial of the warp's 32 x 64 block (lane = row, v = 64
+// accumulator columns), alpha * acc as fp32, through shared memory: every
+// lane writes its row's values, then the warp stores the block one row at a
+// time, two columns per lane, so one store instruction covers 256 contiguous
+// bytes of one row instead of 16 bytes of each of 32 rows (store_partial_64).
+// stg: this warp's STG_WARP_BYTES of idle shared memory; rows: valid rows
+// from row0 (1..32).
+__device__ __forceinline__ void store_partial_staged(const Params &p, int split, float *stg, const float *alpha,
+                                                     int lane, int32_t rows, int32_t row0, int32_t col0,
+                                                     const uint32_t (&v)[64])
+{
+    float *my = stg + lane * STG_LD;
+#pragma unroll
+    for (int j = 0; j < 64; j += 4) {
+        const float4 a = *reinterpret_cast<const float4 *>(&alpha[j]);
+        *reinterpret_cast<float4 *>(my + j) =
+            make_float4(__fmul_rn(__uint_as_float(v[j]), a.x), __fmul_rn(__uint_as_float(v[j + 1]), a.y),
+                        __fmul_rn(__uint_as_float(v[j + 2]), a.z), __fmul_rn(__uint_as_float(v[j + 3]), a.w));
+    }
+    __syncwarp();
+    const int32_t c = col0 + 2 * lane;
+    const bool pairs = (p.N & 1) == 0;
+    float *base = p.partial + static_cast<int64_t>(split) * p.M * p.N;
+    for (int r = 0; r < rows; ++r) {
+        const float2 x = *reinterpret_cast<const float2 *>(stg + r * STG_LD + 2 * lane);
+        float *o = base + static_cast<int64_t>(row0 + r) * p.N + c;
+        if (pairs && c + 1 < p.N) {
+            *reinterpret_cast<float2 *>(o) = x;
+        } else {
+            if (c < p.N)
+                o[0] = x.x;
+            if (c + 1 < p.N)
+                o[1] = x.y;
+        }
+    }
+    __syncwarp();  // the block is read before the next one overwrites it
 }
 
 // out[m, n] = round( sum over splits s = 0, 1, ... of partial[s][m][n] ), the
@@ -620,9 +667,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             if (lane == 0)
                 mbar_arrive(smem_u32(&sm->acc_empty));
             const int row = m0 + q * 32 + lane;
-            if (p.splits > 1) {
-                store_partial_64(p, split, alpha, row, n0 + hc * HALF_N, v0);
-                store_partial_64(p, split, alpha + 64, row, n0 + hc * HALF_N + 64, v1);
+            const int col0 = n0 + hc * HALF_N;
+            const int rows = min(32, p.M - (m0 + q * 32));
+            if (p.splits > 1 && p.staged_partials && item + static_cast<int>(gridDim.x) >= p.num_tiles * p.splits) {
+                // This CTA's last work item: its MMAs are complete (acc_full) and the
+                // producers have nothing left to load, so the pipeline ring is idle
+                // and holds each warp's staging rows.
+                float *stg = reinterpret_cast<float *>(smem + (warp - EPI_WARP0) * STG_WARP_BYTES);
+                if (rows > 0 && col0 < p.N) {
+                    store_partial_staged(p, split, stg, alpha, lane, rows, m0 + q * 32, col0, v0);
+                    store_partial_staged(p, split, stg, alpha + 64, lane, rows, m0 + q * 32, col0 + 64, v1);
+                }
+            } else if (p.splits > 1) {
+                store_partial_64(p, split, alpha, row, col0, v0);
+                store_partial_64(p, split, alpha + 64, row, col0 + 64, v1);
             } else {
                 store_64(p, alpha, row, n0 + hc * HALF_N, v0);
                 store_64(p, alpha + 64, row, n0 + hc * HALF_N + 64, v1);

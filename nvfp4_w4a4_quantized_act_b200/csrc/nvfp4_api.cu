@@ -333,10 +333,16 @@ int make_out_map(CUtensorMap *map, void *out, int64_t rows, int64_t cols)
 // The count minimises a cost model fitted to measurements on B200 at M <= 128:
 // a CTA spends about 0.6 us per K stage (its pipeline is latency-bound at
 // these sizes), while each split adds its fp32 partials (M x N x 4 bytes,
-// written with per-row stores and read back, about 1.5 TB/s together) and a
-// fixed cost for the finalize kernel that adds them (about 2 us).
+// written and read back by the finalize kernel) and a fixed cost for that
+// kernel.  Below 64 rows the partials go out with per-row stores (about 1.5
+// TB/s for the write and read together, 2 us fixed); from 64 rows the CTA's
+// last work item stages them through shared memory, a row per store
+// instruction (about 1.3 ns per partial element, 4.5 us fixed: fitted to
+// split counts 1-8 at M = 64 and 128 on the decode shapes, N = 5120 with K
+// = 5120, 6144, 17408 and N = 14432 with K = 5120).
 constexpr int kSplitKMax = 8;
 constexpr int kSplitKSms = 148;
+constexpr int64_t kStagedPartialRows = 64;
 
 int splitk_count(int64_t M, int64_t N, int64_t K)
 {
@@ -348,11 +354,12 @@ int splitk_count(int64_t M, int64_t N, int64_t K)
     const int64_t s_max = std::min<int64_t>({kSplitKMax, kt_total, std::max<int64_t>(1, kSplitKSms / tiles)});
     int64_t best = 1;
     double best_ns = 600.0 * static_cast<double>(kt_total);
+    const bool staged = M >= kStagedPartialRows;
     for (int64_t want = 2; want <= s_max; ++want) {
         const int64_t kps = cdiv(kt_total, want);
         const int64_t S = cdiv(kt_total, kps);
-        const double ns = 600.0 * static_cast<double>(kps) +
-                          static_cast<double>(S * M * N) * 8.0 / 1500.0 + 2000.0;
+        const double elems = static_cast<double>(S * M * N);
+        const double ns = 600.0 * static_cast<double>(kps) + (staged ? elems * 1.3e-3 + 4500.0 : elems * 8.0 / 1500.0 + 2000.0);
         if (ns < best_ns) {
             best_ns = ns;
             best = S;
@@ -413,6 +420,7 @@ int run_gemm(DeviceState *d, const uint8_t *a_codes, const uint8_t *a_sf, const 
             p.splits = S;
             p.kt_per_split = static_cast<int32_t>(cdiv(p.kt_total, S));
             p.partial = partial;
+            p.staged_partials = M >= kStagedPartialRows ? 1 : 0;
         }
     }
     p.w_early = (w_early && !use_pair) ? 1 : 0;

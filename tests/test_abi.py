@@ -57,11 +57,12 @@ def _act_bytes(M, K):
     (16, 5120, 5120, 5),     # 20 tiles, 20 stages: 5 splits of 4 stages
     (1, 1024, 5120, 7),      # 4 tiles: 7 splits of <= 3 stages (8 would leave 3 per split too)
     (3, 1000, 5120, 7),      # ragged N
-    (128, 1280, 17408, 7),   # 68 stages: 7 splits of <= 10
+    (128, 1280, 17408, 8),   # 68 stages, 5 tiles: 8 splits of <= 9 (staged partials from 64 rows)
     (16, 16480, 5120, 2),    # 65 tiles: at most 148 // 65 = 2
     (64, 16480, 5120, 1),    # the partials would cost more than the stages saved
-    (128, 5120, 5120, 1),
-    (64, 5120, 5120, 3),
+    (128, 5120, 5120, 4),    # staged partials: 4 splits of 5 stages
+    (64, 5120, 5120, 5),     # staged partials: 5 splits of 4 stages
+    (33, 5120, 5120, 4),     # per-row partials below 64 rows
     (128, 34816, 5120, 1),   # 136 tiles fill the GPU: no split
     (16, 5120, 256, 1),      # one stage of K: no split
     (129, 5120, 5120, 1),    # more than one 128-row block: CTA-pair GEMM, no split

@@ -28,6 +28,9 @@ CASES = [
     (128, 1280, 17408, None),
     (100, 5120, 2048, [4096, 1024]),
     (3, 1002, 5120, [500, 502]),  # N % 4 != 0: scalar partial and output stores
+    # from 64 rows the partials go through shared memory, a row per store:
+    (64, 5120, 6144, None),       # 6 splits, two-column stores
+    (100, 1001, 5120, [500, 501]),  # 7 splits, odd N (one-column stores), 4 rows in the last lane quarter
 ]
 
 
