@@ -611,7 +611,7 @@ def decode_roofline(stack, pk, pk_kind, token_counts=(1, 16, 64, 128)):
     from nvfp4_w4a4_quantized_act_b200 import ops
     dev = stack.X.device
     wbytes = sum(qw.codes.numel() + qw.sf.numel() for qs in stack.weights for qw in qs)
-    res = {"kernel": "split-K linear chain (amax + quantize + gemm_nvf4_kernel split-K + split sum) per linear; "
+    res = {"kernel": "split-K linear chain (quantize with its amax + gemm_nvf4_kernel split-K + split sum) per linear; "
                      "gate/up with SwiGLU, down on its quantized h",
            "bound": "hbm", "unit": "GB/s", "peak": pk["hbm_gbs"], "peak_basis": pk_kind,
            "weight_bytes_per_step": int(wbytes), "linears_per_step": 256, "steps": {}}
