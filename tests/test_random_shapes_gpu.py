@@ -1,0 +1,49 @@
+"""nvfp4_linear_fused on seeded random shapes against the oracle: M from one
+row to more than two CTA-pair tiles (split-K with per-row and with staged
+partials, the single-CTA and the CTA-pair GEMM), ragged N, K of one to forty
+64-wide steps, one to four module segments of random widths.  Each case runs
+the bf16 and the fp32 output, checks the activation's codes, scales and
+global scale and the weight's bit for bit, compares sampled outputs (with
+every tail and segment-boundary column of a few rows) with the oracle at
+1e-5 sum|a*b| + 1e-6, and checks that no byte around the outputs and the
+workspace was written."""
+import numpy as np
+import pytest
+
+from nvfp4_w4a4_quantized_act_b200 import workloads as wl
+from nvfp4_testutil import full_size_check
+
+pytestmark = pytest.mark.gpu
+
+
+def _cases(n=24, seed=2026):
+    rng = np.random.default_rng(seed)
+    out = []
+    for i in range(n):
+        # rows: a third decode-sized, a third around the 64-row staged split-K
+        # threshold and the 128-row single-CTA limit, a third CTA-pair sized
+        band = i % 3
+        if band == 0:
+            M = int(rng.integers(1, 40))
+        elif band == 1:
+            M = int(rng.integers(56, 140))
+        else:
+            M = int(rng.integers(129, 600))
+        K = 64 * int(rng.integers(1, 41))
+        N = int(rng.integers(2, 3000))
+        nseg = int(min(N, rng.integers(1, 5)))
+        cuts = np.sort(rng.choice(np.arange(1, N), size=nseg - 1, replace=False)) if nseg > 1 else []
+        edges = [0, *[int(c) for c in cuts], N]
+        widths = [b - a for a, b in zip(edges[:-1], edges[1:])]
+        out.append((M, N, K, widths, 100 + i))
+    return out
+
+
+@pytest.mark.parametrize("M,N,K,widths,seed", _cases())
+def test_random_shape_linear_fused(M, N, K, widths, seed):
+    X = wl.activation_normal(M, K, seed, n_outliers=min(4, K // 16))
+    sig = [0.005 * (1.0 + 3.0 * ((seed * 7 + j) % 4)) for j in range(len(widths))]
+    W = np.concatenate([wl.weight_normal(w, K, s, seed * 10 + j).float().numpy() for j, (w, s) in
+                        enumerate(zip(widths, sig))], 0)
+    ratio = full_size_check(X, wl.to_bf16(W), wl.segments_from_widths(widths), seed)
+    assert ratio <= 1.0
