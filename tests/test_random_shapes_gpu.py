@@ -1,17 +1,26 @@
-"""nvfp4_linear_fused on seeded random shapes against the oracle: M from one
-row to more than two CTA-pair tiles (split-K with per-row and with staged
-partials, the single-CTA and the CTA-pair GEMM), ragged N, K of one to forty
-64-wide steps, one to four module segments of random widths.  Each case runs
-the bf16 and the fp32 output, checks the activation's codes, scales and
-global scale and the weight's bit for bit, compares sampled outputs (with
-every tail and segment-boundary column of a few rows) with the oracle at
-1e-5 sum|a*b| + 1e-6, and checks that no byte around the outputs and the
-workspace was written."""
+"""Seeded random shapes against the oracle.
+
+nvfp4_linear_fused: M from one row to more than two CTA-pair tiles (split-K
+with per-row and with staged partials, the single-CTA and the CTA-pair
+GEMM), ragged N, K of one to forty 64-wide steps, one to four module
+segments of random widths.  Each case runs the bf16 and the fp32 output,
+checks the activation's codes, scales and global scale and the weight's bit
+for bit, compares sampled outputs (with every tail and segment-boundary
+column of a few rows) with the oracle at 1e-5 sum|a*b| + 1e-6, and checks
+that no byte around the outputs and the workspace was written.
+
+nvfp4_linear_swiglu: random M, K and F (a multiple of 128) through both
+gated kernels, h against silu(gate) up of the oracle's GEMM and h's codes,
+scales and global scale bit for bit.  nvfp4_quantize_act: random rows and K
+(a multiple of 16), codes, scales (padding included) and global scale bit
+for bit."""
 import numpy as np
 import pytest
 
 from nvfp4_w4a4_quantized_act_b200 import workloads as wl
 from nvfp4_testutil import full_size_check
+from test_quant_gpu import _assert_same
+from test_swiglu_fused_gpu import _check as _check_swiglu, _gate_up
 
 pytestmark = pytest.mark.gpu
 
@@ -47,3 +56,31 @@ def test_random_shape_linear_fused(M, N, K, widths, seed):
                         enumerate(zip(widths, sig))], 0)
     ratio = full_size_check(X, wl.to_bf16(W), wl.segments_from_widths(widths), seed)
     assert ratio <= 1.0
+
+
+def _gated_cases(n=8, seed=77):
+    rng = np.random.default_rng(seed)
+    out = []
+    for i in range(n):
+        M = int(rng.integers(1, 128)) if i % 2 == 0 else int(rng.integers(129, 420))
+        K = 64 * int(rng.integers(1, 25))
+        F = 128 * int(rng.integers(1, 9))
+        out.append((M, K, F, bool(i % 4 == 1), 300 + i))
+    return out
+
+
+@pytest.mark.parametrize("M,K,F,single_cta,seed", _gated_cases())
+def test_random_shape_linear_swiglu(M, K, F, single_cta, seed):
+    X = wl.activation_normal(M, K, seed, n_outliers=min(4, K // 16))
+    W = _gate_up(F, K, seed + 1)
+    _check_swiglu(M, K, F, X, W, np.arange(M), np.arange(F), single_cta)
+
+
+def _quant_cases(n=12, seed=91):
+    rng = np.random.default_rng(seed)
+    return [(int(rng.integers(1, 700)), 16 * int(rng.integers(1, 200)), 500 + i) for i in range(n)]
+
+
+@pytest.mark.parametrize("M,K,seed", _quant_cases())
+def test_random_shape_quantize_act(M, K, seed):
+    _assert_same(wl.activation_normal(M, K, seed, n_outliers=min(4, K // 16), scale=30.0))
