@@ -9,6 +9,11 @@ for bit, compares sampled outputs (with every tail and segment-boundary
 column of a few rows) with the oracle at 1e-5 sum|a*b| + 1e-6, and checks
 that no byte around the outputs and the workspace was written.
 
+Decode sizes with split-K: M up to 128 with K of 1536 to 17408, so that the
+split count is 3-8 for most cases, per-row partials below 64 rows and
+staged ones above; every row against the oracle, bf16 = RNE(fp32), run to
+run and pre-quantized forms bit-identical (the decode suite's checker).
+
 nvfp4_linear_swiglu: random M, K and F (a multiple of 128) through both
 gated kernels, h against silu(gate) up of the oracle's GEMM and h's codes,
 scales and global scale bit for bit.  nvfp4_quantize_act: random rows and K
@@ -19,6 +24,7 @@ import pytest
 
 from nvfp4_w4a4_quantized_act_b200 import workloads as wl
 from nvfp4_testutil import full_size_check
+from test_decode_gpu import test_decode_linear_matches_oracle as decode_check
 from test_quant_gpu import _assert_same
 from test_swiglu_fused_gpu import _check as _check_swiglu, _gate_up
 
@@ -84,3 +90,23 @@ def _quant_cases(n=12, seed=91):
 @pytest.mark.parametrize("M,K,seed", _quant_cases())
 def test_random_shape_quantize_act(M, K, seed):
     _assert_same(wl.activation_normal(M, K, seed, n_outliers=min(4, K // 16), scale=30.0))
+
+
+def _decode_cases(n=16, seed=4242):
+    rng = np.random.default_rng(seed)
+    out = []
+    for i in range(n):
+        M = int(rng.integers(1, 64)) if i % 2 == 0 else int(rng.integers(64, 129))
+        K = 64 * int(rng.integers(24, 273))
+        N = int(rng.integers(64, 6000))
+        nseg = int(rng.integers(1, 4))
+        cuts = np.sort(rng.choice(np.arange(1, N), size=nseg - 1, replace=False)) if nseg > 1 else []
+        edges = [0, *[int(c) for c in cuts], N]
+        widths = [b - a for a, b in zip(edges[:-1], edges[1:])] if nseg > 1 else None
+        out.append((M, N, K, widths))
+    return out
+
+
+@pytest.mark.parametrize("M,N,K,widths", _decode_cases())
+def test_random_shape_decode_split_k(M, N, K, widths):
+    decode_check(M, N, K, widths)
