@@ -258,7 +258,9 @@ def test_on_grid_blocks_are_reproduced_exactly():
 # ------------------------------------------------------- scale-factor layout
 
 def test_sf_layout_is_bijection_of_512_byte_tiles():
-    for rows, K in [(1, 64), (130, 256), (256, 320), (64, 16)]:
+    # (300, 80) and (260, 48): several row tiles with K / 16 not a multiple
+    # of 4, where the padded K-tile count sets the row tiles' stride
+    for rows, K in [(1, 64), (130, 256), (256, 320), (64, 16), (300, 80), (260, 48)]:
         total = oracle.sf_bytes(rows, K)
         rpad = (rows + 127) // 128 * 128
         cpad = (K // 16 + 3) // 4 * 4
@@ -296,7 +298,7 @@ def _documented_sf_positions(rows, K):
 
 
 def test_sf_layout_matches_documented_interleave():
-    for rows, K in [(1, 64), (128, 64), (130, 256), (300, 1344), (64, 16)]:
+    for rows, K in [(1, 64), (128, 64), (130, 256), (300, 1344), (64, 16), (300, 80), (260, 48)]:
         pos = _documented_sf_positions(rows, K)
         got = np.array([[oracle.sf_offset(r, c, K) for c in range(pos.shape[1])] for r in range(pos.shape[0])])
         assert np.array_equal(got, pos), (rows, K)

@@ -54,17 +54,22 @@ MUTANTS = {
     # scale-factor layout
     "sf_tile_row_major": (C, "(rr % 32) * 16 + (rr / 32) * 4 + (c % 4)", "(rr / 4) * 16 + (rr % 4) * 4 + (c % 4)"),
     "sf_tiles_unpadded_k": (C, "int64_t cpad = (K / 16 + 3) / 4 * 4;", "int64_t cpad = K / 16;"),
+    "sf_tile_stride_unpadded": (C, "int64_t ct_count = (K / 16 + 3) / 4;", "int64_t ct_count = K / 64;"),
     # dequantization and GEMM
     "dequant_scale_per_32": (C, "double s = oracle_e4m3_decode(scales[r * nb + k / 16]);",
                              "double s = oracle_e4m3_decode(scales[r * nb + k / 32]);"),
     "gemm_a_nibbles_swapped": (C, "int ac = (k & 1) ? (ab >> 4) : (ab & 15);", "int ac = (k & 1) ? (ab & 15) : (ab >> 4);"),
     "gemm_w_takes_g_a": (C, "* (double)g_w_row[n];", "* (double)g_a;"),
     "gemm_bound_signed": (C, "bound += fabs(a * w);", "bound += a * w;"),
+    "sampled_w_row_from_m": (C, "uint8_t wb = w_codes[n * (K / 2) + k / 2];", "uint8_t wb = w_codes[m * (K / 2) + k / 2];"),
+    "dequant_nibbles_swapped": (C, "int c = (k & 1) ? (byte >> 4) : (byte & 15);", "int c = (k & 1) ? (byte & 15) : (byte >> 4);"),
+    "block_stride_8": (C, "const uint16_t *blk = x + r * ld + b * 16;", "const uint16_t *blk = x + r * ld + b * 8;"),
     # MLP intermediate and bf16 rounding
     "silu_exp_sign": (C, "double s = gv / (1.0 + exp(-gv));", "double s = gv / (1.0 + exp(gv));"),
     "swiglu_up_is_gate": (C, "gate_up[r * ld + F + j]", "gate_up[r * ld + j]"),
     "bf16_ties_away": (C, "double r = nearbyint(q);", "double r = round(q);"),
     "bf16_one_bit_short": (C, "int ulp_exp = (e - 1) - 7;", "int ulp_exp = (e - 1) - 6;"),
+    "bf16_subnormals_flushed_early": (C, "if (ulp_exp < -133)\n        ulp_exp = -133;", "if (ulp_exp < -126)\n        ulp_exp = -126;"),
     # FP8 KV cache
     "kv_scale_240": (C, "float s = amax / 448.0f;", "float s = amax / 240.0f;"),
     "kv_drops_sign": (C, "return signbit(y) ? (m | 0x80) : m;", "return m;"),
