@@ -236,6 +236,51 @@ def test_exhaustive_bf16_against_numpy_pipeline():
         assert np.array_equal(np.signbit(got), np.signbit(want))
 
 
+def _e4m3_of_f32(s32: np.ndarray) -> np.ndarray:
+    """E4M3 byte of non-negative fp32 values: torch's round-to-nearest-even
+    conversion below 464 (the midpoint above 448), 448 (0x7E) from there."""
+    out = np.full(s32.shape, 0x7E, dtype=np.uint8)
+    low = s32 < 464
+    out[low] = _torch_e4m3(s32[low])
+    return out
+
+
+def test_scale_byte_follows_the_r2_operation_order():
+    """The block scale byte is E4M3(fl32(fl32(bamax / 6) / g)) (R2).  Global
+    scales are chosen so that the scale lands within a few fp32 ulps of an
+    E4M3 rounding midpoint, where forming it as bamax / fl32(6 g) instead
+    rounds to the other neighbour for some pairs; every pair is checked on
+    a block with one live element against numpy fp32 arithmetic and torch's
+    E4M3 conversion."""
+    rng = np.random.default_rng(5)
+    tab = oracle.e4m3_table()[:0x7F].astype(np.float64)
+    mids = ((tab[:-1] + tab[1:]) / 2)[8:]                    # normal-range midpoints
+    b_bits = rng.integers(0x3C00, 0x4700, 400).astype(np.uint16)  # bf16 block amax, ~2^-7 .. 2^15
+    bam = oracle.bf16_bits_to_f32(b_bits).astype(np.float32)
+    pairs_b, pairs_g = [], []
+    for m in mids:
+        t = (bam / np.float32(6)).astype(np.float32)
+        g0 = (t / np.float32(m)).astype(np.float32)
+        for g in (g0, np.nextafter(g0, np.float32(0)), np.nextafter(g0, np.float32(np.inf))):
+            ok = np.isfinite(g) & (g > 0)
+            pairs_b.append(b_bits[ok])
+            pairs_g.append(g[ok])
+    pb = np.concatenate(pairs_b)
+    pg = np.concatenate(pairs_g).astype(np.float32)
+    bv = oracle.bf16_bits_to_f32(pb).astype(np.float32)
+    s32 = ((bv / np.float32(6)).astype(np.float32) / pg).astype(np.float32)
+    alt = (bv / (np.float32(6) * pg).astype(np.float32)).astype(np.float32)
+    want = _e4m3_of_f32(s32)
+    discriminating = want != _e4m3_of_f32(alt)
+    assert discriminating.sum() > 0  # the pairs do tell the two orders apart
+    pick = np.unique(np.concatenate([np.flatnonzero(discriminating), rng.integers(0, len(pb), 2000)]))
+    for i in pick:
+        blk = np.zeros((1, 16), dtype=np.uint16)
+        blk[0, 3] = pb[i]
+        _, scales = oracle.quantize(blk, pg[i])
+        assert scales[0, 0] == want[i], (hex(pb[i]), float(pg[i]))
+
+
 def test_on_grid_blocks_are_reproduced_exactly():
     """g = 1 and blocks whose largest code is 6: quantize(dequant(q)) == q
     and the reconstruction error is zero (scale identity)."""

@@ -36,6 +36,10 @@ MUTANTS = {
     "block_scale_over_4": (C, "float t = bamax / 6.0f;", "float t = bamax / 4.0f;"),
     "block_scale_times_g": (C, "float s32 = t / g;", "float s32 = t * g;"),
     "divisor_without_g": (C, "float d = s * g;", "float d = s;"),
+    "scale_product_order": (C, "float t = bamax / 6.0f;\n            float s32 = t / g;",
+                            "float t = bamax;\n            float s32 = t / (6.0f * g);"),
+    "quotient_two_divisions": (C, "float y = xv / d;", "float y = xv / s / g;"),
+    "kv_scale_nvfp4_divisor": (C, "float s = amax / 448.0f;", "float s = amax / 2688.0f;"),
     "multiply_not_divide": (C, "float y = xv / d;", "float y = xv * d;"),
     "zero_block_drops_sign": (C, "c[j] = signbit(xv) ? 8 : 0;", "c[j] = 0;"),
     "nibbles_swapped": (C, "(uint8_t)(c[0] | (c[1] << 4))", "(uint8_t)(c[1] | (c[0] << 4))"),
@@ -51,6 +55,9 @@ MUTANTS = {
     "e4m3_bias_8": (C, "v = (1.0 + m / 8.0) * ldexp(1.0, e - 7);", "v = (1.0 + m / 8.0) * ldexp(1.0, e - 8);"),
     "e4m3_subnormal_exp": (C, "v = (m / 8.0) * ldexp(1.0, -6);", "v = (m / 8.0) * ldexp(1.0, -7);"),
     "e4m3_ieee_top_binade": (C, "if (e == 15 && m == 7)", "if (e == 15)"),
+    "e4m3_grid_without_448": (C, "return nearest_even_code(a, vals, codes, 127);",
+                              "return nearest_even_code(a, vals, codes, 126);"),
+    "e2m1_saturates_from_5": (C, "if (a >= 6.0)\n        mag = 7;", "if (a >= 5.0)\n        mag = 7;"),
     # scale-factor layout
     "sf_tile_row_major": (C, "(rr % 32) * 16 + (rr / 32) * 4 + (c % 4)", "(rr / 4) * 16 + (rr % 4) * 4 + (c % 4)"),
     "sf_tiles_unpadded_k": (C, "int64_t cpad = (K / 16 + 3) / 4 * 4;", "int64_t cpad = K / 16;"),
